@@ -1,0 +1,562 @@
+/*
+ * sphkv_oracle.c -- plain fp64 CPU oracle for Spherical KV.
+ *
+ * TEST INFRASTRUCTURE ONLY.  The test suite, the smoke check and the CPU
+ * baseline leg of the benchmark are the only callers of this library; the
+ * product path never loads it.  It shares no code, header, table or helper
+ * with the CUDA library.
+ *
+ * What it follows.  "SPHERICAL KV: Angle-Domain Attention and Rate-Distortion
+ * Retention for Efficient Long-Context Inference" (arXiv 2605.18856), Abstract
+ * and AI Summary:
+ *   - ADA keeps every key as a scalar radius plus compact angle codes (a point
+ *     on the hypersphere) and gets the attention logits from those codes;
+ *   - RDR chooses keep/drop and a precision tier for each unit under a fixed
+ *     byte budget, as a rate-distortion problem, so that pages are
+ *     tier-homogeneous.
+ * The pages fix no formula, grid, bit width or layout.  The format written out
+ * here is the one this project fixes: a recursive-polar (binary-tree)
+ * parameterisation with d/2 leaf pair angles and d/2-1 upper angles, three
+ * tiers (T1 8/8 bits + int8 V, T2 4/6 bits + int4 V, T3 3/4 bits + int4 V),
+ * 16-token pages and a Lagrangian bisection for RDR.  Every reading of a point
+ * the pages leave open is listed in the project's design notes.
+ *
+ * How.  Plain loops in fp64, compiled with -ffp-contract=off so no product is
+ * ever fused into an add.  Attention is done the slow, obvious way: decode the
+ * codes to a dense fp64 key, then dense softmax attention.  The bottom-up
+ * logit tree is present only so the tests can check it against that.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_PAGE 16
+#define ORC_D 128 /* head size of the packed page format */
+
+/* ---------------------------------------------------------------- fp16 -- */
+
+/* Round a double to IEEE binary16, round-half-to-even, one rounding step. */
+uint16_t orc_f64_to_f16(double x)
+{
+    uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    double a = fabs(x);
+    if (isnan(x)) return 0x7e00u;
+    if (isinf(x)) return (uint16_t)(sign | 0x7c00u);
+    if (a == 0.0) return sign;
+    int e;
+    (void)frexp(a, &e);          /* a = m * 2^e, m in [0.5, 1) */
+    int E = e - 1;               /* a in [2^E, 2^(E+1)) */
+    if (E < -14) E = -14;        /* subnormal range shares the 2^-24 quantum */
+    double quantum = ldexp(1.0, E - 10);
+    double n = rint(a / quantum); /* exact scaling by a power of two, then RNE */
+    if (n >= 2048.0) { E += 1; n = n / 2.0; }
+    if (E > 15) return (uint16_t)(sign | 0x7c00u);
+    if (n < 1024.0) return (uint16_t)(sign | (uint16_t)n); /* subnormal */
+    return (uint16_t)(sign | (uint16_t)(((E + 15) << 10) | ((int)n - 1024)));
+}
+
+double orc_f16_to_f64(uint16_t h)
+{
+    int s = (h >> 15) & 1, ex = (h >> 10) & 0x1f, m = h & 0x3ff;
+    double v;
+    if (ex == 0) v = ldexp((double)m, -24);
+    else if (ex == 31) v = m ? NAN : INFINITY;
+    else v = ldexp((double)(m + 1024), ex - 25);
+    return s ? -v : v;
+}
+
+/* ------------------------------------------------------------- tiers -- */
+
+/* Tier index 1..3 -> (b_leaf, b_up, v_bits).  0 is "drop". */
+static const int ORC_BLEAF[4] = {0, 8, 4, 3};
+static const int ORC_BUP[4] = {0, 8, 6, 4};
+static const int ORC_VBITS[4] = {0, 8, 4, 4};
+
+/* Byte sizes of one token row of each field in a page of the given tier. */
+static int leaf_row_bytes(int t) { return (ORC_D / 2) * ORC_BLEAF[t] / 8; }
+static int up_row_bytes(int t) { return ((ORC_D / 2 - 1) * ORC_BUP[t] + 127) / 128 * 16; }
+static int v_row_bytes(int t) { return ORC_D * ORC_VBITS[t] / 8; }
+
+/* Field offsets inside a page: r[16] fp16, vscale[16] fp16, leaf rows, upper
+ * rows, value rows. */
+static int off_leaf(int t) { (void)t; return 2 * ORC_PAGE * 2; }
+static int off_up(int t) { return off_leaf(t) + ORC_PAGE * leaf_row_bytes(t); }
+static int off_v(int t) { return off_up(t) + ORC_PAGE * up_row_bytes(t); }
+
+int orc_page_bytes(int t)
+{
+    if (t < 1 || t > 3) return 0;
+    return off_v(t) + ORC_PAGE * v_row_bytes(t);
+}
+
+/* ------------------------------------------------------------ encode -- */
+
+/* Leaf angle code.  phi = atan2(y, x) in (-pi, pi]; the grid is periodic with
+ * 2^b points at c * 2pi / 2^b; rounding to nearest (ties to even); a zero pair
+ * gets code 0. */
+static int leaf_code(double x, double y, int b)
+{
+    long M = 1L << b;
+    if (x == 0.0 && y == 0.0) return 0;
+    double phi = atan2(y, x);
+    double t = rint((phi * (double)M) / (2.0 * M_PI));
+    long c = (long)t;
+    c = ((c % M) + M) % M;
+    return (int)c;
+}
+
+/* Upper angle code.  psi = atan2(|right|, |left|) in [0, pi/2]; the grid
+ * includes both ends: c * (pi/2) / (2^b - 1), c = 0 .. 2^b - 1. */
+static int upper_code(double ss_left, double ss_right, int b)
+{
+    long top = (1L << b) - 1;
+    double nl = sqrt(ss_left), nr = sqrt(ss_right);
+    double psi = (nl == 0.0 && nr == 0.0) ? 0.0 : atan2(nr, nl);
+    double t = rint((psi * (double)top) / M_PI_2);
+    if (t < 0.0) t = 0.0;
+    if (t > (double)top) t = (double)top;
+    return (int)t;
+}
+
+/* Encode one token of one head.  k, v: [d] fp64 (exact copies of the bf16 or
+ * fp32 inputs).  leaf: [d/2] codes, up: [d/2-1] codes in level order (level 1
+ * parents of leaves (2m, 2m+1) first, the root last).  Returns 0, or 1 when
+ * the radius or the value scale overflows fp16. */
+static int encode_one(int d, const double* k_in, const double* v, int b_leaf, int b_up,
+                      int v_bits, uint8_t* leaf, uint8_t* up, uint16_t* r16, uint16_t* s16,
+                      int8_t* vq, double* work)
+{
+    int L = d / 2;
+    double* k = work;          /* [d] */
+    double* ss = work + d;     /* [2L - 1]: leaves then upper nodes, level order */
+    for (int i = 0; i < d; ++i) k[i] = k_in[i] + 0.0; /* -0 -> +0 */
+    for (int j = 0; j < L; ++j) {
+        double x = k[2 * j], y = k[2 * j + 1];
+        ss[j] = x * x + y * y;
+        leaf[j] = (uint8_t)leaf_code(x, y, b_leaf);
+    }
+    /* upper nodes: children of level-(l) node m are nodes 2m, 2m+1 of level l-1 */
+    int child = 0, node = L, width = L / 2, u = 0;
+    while (width >= 1) {
+        for (int m = 0; m < width; ++m) {
+            double sl = ss[child + 2 * m], sr = ss[child + 2 * m + 1];
+            ss[node + m] = sl + sr;
+            up[u++] = (uint8_t)upper_code(sl, sr, b_up);
+        }
+        child = node;
+        node += width;
+        width /= 2;
+    }
+    int bad = 0;
+    double r = sqrt(ss[2 * L - 2]);
+    *r16 = orc_f64_to_f16(r);
+    if ((*r16 & 0x7c00u) == 0x7c00u) bad = 1;
+
+    double Q = (v_bits == 8) ? 127.0 : 7.0;
+    double a = 0.0;
+    for (int c = 0; c < d; ++c) a = fmax(a, fabs(v[c]));
+    *s16 = orc_f64_to_f16(a / Q);
+    if ((*s16 & 0x7c00u) == 0x7c00u) bad = 1;
+    double s = orc_f16_to_f64(*s16);
+    for (int c = 0; c < d; ++c) {
+        double t = (s == 0.0) ? 0.0 : rint(v[c] / s);
+        if (t > Q) t = Q;
+        if (t < -Q) t = -Q;
+        vq[c] = (int8_t)t;
+    }
+    return bad;
+}
+
+/* Encode n tokens (rows of K and V, each [d]).  Returns the number of tokens
+ * whose radius or value scale overflowed fp16. */
+int64_t orc_encode_tokens(int64_t n, int d, const double* K, const double* V, int b_leaf,
+                          int b_up, int v_bits, uint8_t* leaf, uint8_t* up, uint16_t* r16,
+                          uint16_t* s16, int8_t* vq)
+{
+    int64_t bad = 0;
+    int L = d / 2;
+#pragma omp parallel reduction(+ : bad)
+    {
+        double* work = (double*)malloc(sizeof(double) * (size_t)(3 * d));
+#pragma omp for schedule(static)
+        for (int64_t i = 0; i < n; ++i)
+            bad += encode_one(d, K + i * d, V + i * d, b_leaf, b_up, v_bits, leaf + i * L,
+                              up + i * (L - 1), r16 + i, s16 + i, vq + i * d, work);
+        free(work);
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------------ decode -- */
+
+static double leaf_angle(int c, int b) { return (2.0 * M_PI * (double)c) / (double)(1L << b); }
+static double upper_angle(int c, int b) { return (M_PI_2 * (double)c) / (double)((1L << b) - 1); }
+
+/* Unit direction from the codes, top-down: the root has weight 1, a left child
+ * gets w*cos(psi), a right child w*sin(psi); leaf j gives
+ * (w_j cos(phi_j), w_j sin(phi_j)). */
+static void unit_vector(int d, const uint8_t* leaf, const uint8_t* up, int b_leaf, int b_up,
+                        double* u, double* w)
+{
+    int L = d / 2;
+    /* w holds node weights in level order (leaves 0..L-1, upper nodes after). */
+    w[2 * L - 2] = 1.0;
+    int node = 2 * L - 2, width = 1;
+    /* walk levels from the root down; upper node index in up[] == node - L */
+    while (width < L) {
+        int child = node - 2 * width; /* first node of the level below */
+        for (int m = 0; m < width; ++m) {
+            double psi = upper_angle(up[node - L + m], b_up);
+            double wn = w[node + m];
+            w[child + 2 * m] = wn * cos(psi);
+            w[child + 2 * m + 1] = wn * sin(psi);
+        }
+        node = child;
+        width *= 2;
+    }
+    for (int j = 0; j < L; ++j) {
+        double phi = leaf_angle(leaf[j], b_leaf);
+        u[2 * j] = w[j] * cos(phi);
+        u[2 * j + 1] = w[j] * sin(phi);
+    }
+}
+
+/* k_hat = r_hat * u_hat for one token; w is [d] scratch. */
+static void decode_key_one(int d, const uint8_t* leaf, const uint8_t* up, uint16_t r16,
+                           int b_leaf, int b_up, double* khat, double* w)
+{
+    unit_vector(d, leaf, up, b_leaf, b_up, khat, w);
+    double r = orc_f16_to_f64(r16);
+    for (int c = 0; c < d; ++c) khat[c] = r * khat[c];
+}
+
+/* k_hat = r_hat * u_hat for n tokens. */
+void orc_decode_keys(int64_t n, int d, const uint8_t* leaf, const uint8_t* up,
+                     const uint16_t* r16, int b_leaf, int b_up, double* khat)
+{
+    int L = d / 2;
+#pragma omp parallel
+    {
+        double* w = (double*)malloc(sizeof(double) * (size_t)(2 * L));
+#pragma omp for schedule(static)
+        for (int64_t i = 0; i < n; ++i)
+            decode_key_one(d, leaf + i * L, up + i * (L - 1), r16[i], b_leaf, b_up,
+                           khat + i * d, w);
+        free(w);
+    }
+}
+
+/* v_hat = code * scale for n tokens. */
+void orc_decode_values(int64_t n, int d, const int8_t* vq, const uint16_t* s16, double* vhat)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        double s = orc_f16_to_f64(s16[i]);
+        for (int c = 0; c < d; ++c) vhat[i * d + c] = (double)vq[i * d + c] * s;
+    }
+}
+
+/* Bottom-up angle-domain logit: leaf S_j = q_2j cos(phi_j) + q_2j+1 sin(phi_j),
+ * node S = cos(psi) S_left + sin(psi) S_right, logit = r_hat S_root / sqrt(d).
+ * Used only by the tests, to check it against q . decode(codes) / sqrt(d). */
+void orc_tree_logits(int64_t n, int d, const uint8_t* leaf, const uint8_t* up,
+                     const uint16_t* r16, int b_leaf, int b_up, const double* q,
+                     double* logits)
+{
+    int L = d / 2;
+    double* S = (double*)malloc(sizeof(double) * (size_t)(2 * L));
+    for (int64_t i = 0; i < n; ++i) {
+        const uint8_t* lc = leaf + i * L;
+        const uint8_t* uc = up + i * (L - 1);
+        for (int j = 0; j < L; ++j) {
+            double phi = leaf_angle(lc[j], b_leaf);
+            S[j] = q[2 * j] * cos(phi) + q[2 * j + 1] * sin(phi);
+        }
+        int child = 0, node = L, width = L / 2;
+        while (width >= 1) {
+            for (int m = 0; m < width; ++m) {
+                double psi = upper_angle(uc[node - L + m], b_up);
+                S[node + m] = cos(psi) * S[child + 2 * m] + sin(psi) * S[child + 2 * m + 1];
+            }
+            child = node;
+            node += width;
+            width /= 2;
+        }
+        logits[i] = orc_f16_to_f64(r16[i]) * S[2 * L - 2] / sqrt((double)d);
+    }
+    free(S);
+}
+
+/* --------------------------------------------------------- attention -- */
+
+/* Dense softmax attention of n_q query rows over n_keys (all kept) keys.
+ * logit_t = q . k_t / sqrt(d); out = sum_t e^(l_t - M) v_t / sum_t e^(l_t - M);
+ * lse = M + ln(sum_t e^(l_t - M)).  No keys: out = 0, lse = -inf. */
+void orc_attention(int64_t n_keys, int d, const double* khat, const double* vhat, int n_q,
+                   const double* q, double* out, double* lse)
+{
+    double* l = (double*)malloc(sizeof(double) * (size_t)(n_keys > 0 ? n_keys : 1));
+    double sd = sqrt((double)d);
+    for (int h = 0; h < n_q; ++h) {
+        const double* qh = q + (int64_t)h * d;
+        double* oh = out + (int64_t)h * d;
+        for (int c = 0; c < d; ++c) oh[c] = 0.0;
+        if (n_keys == 0) { lse[h] = -INFINITY; continue; }
+        double M = -INFINITY;
+        for (int64_t t = 0; t < n_keys; ++t) {
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c) dot += qh[c] * khat[t * d + c];
+            l[t] = dot / sd;
+            if (l[t] > M) M = l[t];
+        }
+        double Z = 0.0;
+        for (int64_t t = 0; t < n_keys; ++t) {
+            double e = exp(l[t] - M);
+            Z += e;
+            for (int c = 0; c < d; ++c) oh[c] += e * vhat[t * d + c];
+        }
+        for (int c = 0; c < d; ++c) oh[c] /= Z;
+        lse[h] = M + log(Z);
+    }
+    free(l);
+}
+
+/* -------------------------------------------------------- page format -- */
+
+/* Write the low `bits` bits of `val` into a little-endian, LSB-first bit
+ * stream starting at bit `pos` of `row`. */
+static void put_bits(uint8_t* row, int pos, int bits, unsigned val)
+{
+    for (int i = 0; i < bits; ++i) {
+        int p = pos + i;
+        if ((val >> i) & 1u) row[p >> 3] |= (uint8_t)(1u << (p & 7));
+        else row[p >> 3] &= (uint8_t)~(1u << (p & 7));
+    }
+}
+
+static unsigned get_bits(const uint8_t* row, int pos, int bits)
+{
+    unsigned v = 0;
+    for (int i = 0; i < bits; ++i) {
+        int p = pos + i;
+        v |= (unsigned)((row[p >> 3] >> (p & 7)) & 1u) << i;
+    }
+    return v;
+}
+
+/* Store one token (d = 128) into slot `slot` of a page of tier t (1..3).
+ * Pad bits of the rows are written as zero. */
+void orc_pack_token(int t, int slot, const uint8_t* leaf, const uint8_t* up, uint16_t r16,
+                    uint16_t s16, const int8_t* vq, uint8_t* page)
+{
+    int bl = ORC_BLEAF[t], bu = ORC_BUP[t], vb = ORC_VBITS[t];
+    page[2 * slot] = (uint8_t)(r16 & 0xff);
+    page[2 * slot + 1] = (uint8_t)(r16 >> 8);
+    page[2 * ORC_PAGE + 2 * slot] = (uint8_t)(s16 & 0xff);
+    page[2 * ORC_PAGE + 2 * slot + 1] = (uint8_t)(s16 >> 8);
+    uint8_t* lrow = page + off_leaf(t) + slot * leaf_row_bytes(t);
+    memset(lrow, 0, (size_t)leaf_row_bytes(t));
+    for (int j = 0; j < ORC_D / 2; ++j) put_bits(lrow, j * bl, bl, leaf[j]);
+    uint8_t* urow = page + off_up(t) + slot * up_row_bytes(t);
+    memset(urow, 0, (size_t)up_row_bytes(t));
+    for (int m = 0; m < ORC_D / 2 - 1; ++m) put_bits(urow, m * bu, bu, up[m]);
+    uint8_t* vrow = page + off_v(t) + slot * v_row_bytes(t);
+    memset(vrow, 0, (size_t)v_row_bytes(t));
+    for (int c = 0; c < ORC_D; ++c) put_bits(vrow, c * vb, vb, (unsigned)(vq[c] & ((1 << vb) - 1)));
+}
+
+void orc_unpack_token(int t, int slot, const uint8_t* page, uint8_t* leaf, uint8_t* up,
+                      uint16_t* r16, uint16_t* s16, int8_t* vq)
+{
+    int bl = ORC_BLEAF[t], bu = ORC_BUP[t], vb = ORC_VBITS[t];
+    *r16 = (uint16_t)(page[2 * slot] | (page[2 * slot + 1] << 8));
+    *s16 = (uint16_t)(page[2 * ORC_PAGE + 2 * slot] | (page[2 * ORC_PAGE + 2 * slot + 1] << 8));
+    const uint8_t* lrow = page + off_leaf(t) + slot * leaf_row_bytes(t);
+    for (int j = 0; j < ORC_D / 2; ++j) leaf[j] = (uint8_t)get_bits(lrow, j * bl, bl);
+    const uint8_t* urow = page + off_up(t) + slot * up_row_bytes(t);
+    for (int m = 0; m < ORC_D / 2 - 1; ++m) up[m] = (uint8_t)get_bits(urow, m * bu, bu);
+    const uint8_t* vrow = page + off_v(t) + slot * v_row_bytes(t);
+    for (int c = 0; c < ORC_D; ++c) {
+        int raw = (int)get_bits(vrow, c * vb, vb);
+        if (raw >= (1 << (vb - 1))) raw -= (1 << vb); /* two's complement */
+        vq[c] = (int8_t)raw;
+    }
+}
+
+/* Page-table entry: bits 31..30 tier (0 drop, 1 T1, 2 T2, 3 T3), bits 29..0
+ * the page's index in that tier's pool. */
+void orc_build_page_table(int64_t n_entries, const uint8_t* tiers, const int32_t* perm1,
+                          const int32_t* perm2, const int32_t* perm3, int32_t* table)
+{
+    const int32_t* perm[4] = {NULL, perm1, perm2, perm3};
+    int64_t next[4] = {0, 0, 0, 0};
+    for (int64_t i = 0; i < n_entries; ++i) {
+        int t = tiers[i];
+        if (t == 0) { table[i] = 0; continue; }
+        int64_t k = next[t]++;
+        int64_t phys = perm[t] ? perm[t][k] : k;
+        table[i] = (int32_t)(((uint32_t)t << 30) | (uint32_t)phys);
+    }
+}
+
+/* Decode attention over a paged cache, computed the slow way, for the units
+ * (sequence b, kv head g) listed in sel_b/sel_g.  For each unit: unpack every
+ * kept token (t < seq_len, page not dropped), decode it to a dense fp64 key and
+ * value, then dense softmax attention for the G = H_q / H_kv query heads
+ * h = g*G .. g*G+G-1 (query head h reads kv head h / G).
+ * q: [B][H_q][128]; out: [n_sel][G][128]; lse: [n_sel][G].
+ * page_table: [H_kv][total_pages]; page_offsets: [B+1] (pages of sequence b
+ * are page_offsets[b] .. page_offsets[b+1]-1, for every kv head).
+ * Returns 0, or 6 for an entry whose page index lies outside its pool. */
+int orc_cache_attention(int B, int H_q, int H_kv, int64_t total_pages, const int32_t* page_offsets,
+                        const int32_t* seq_lens, const int32_t* page_table, const uint8_t* pool1,
+                        const uint8_t* pool2, const uint8_t* pool3, const int64_t* pool_pages,
+                        const double* q, int n_sel, const int32_t* sel_b, const int32_t* sel_g,
+                        double* out, double* lse)
+{
+    const uint8_t* pools[4] = {NULL, pool1, pool2, pool3};
+    int G = H_q / H_kv;
+    int status = 0;
+    (void)B;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int s = 0; s < n_sel; ++s) {
+        int b = sel_b[s], g = sel_g[s];
+        int64_t len = seq_lens[b];
+        int64_t first = page_offsets[b];
+        double* K = (double*)malloc(sizeof(double) * (size_t)(len > 0 ? len : 1) * ORC_D);
+        double* V = (double*)malloc(sizeof(double) * (size_t)(len > 0 ? len : 1) * ORC_D);
+        uint8_t leaf[ORC_D / 2], up[ORC_D / 2 - 1];
+        int8_t vq[ORC_D];
+        double w[ORC_D];
+        uint16_t r16, s16;
+        int64_t n = 0;
+        for (int64_t t = 0; t < len; ++t) {
+            int32_t e = page_table[(int64_t)g * total_pages + first + t / ORC_PAGE];
+            int tier = (int)(((uint32_t)e) >> 30);
+            int64_t phys = (int64_t)(((uint32_t)e) & 0x3fffffffu);
+            if (tier == 0) continue;
+            if (phys >= pool_pages[tier - 1]) {
+#pragma omp atomic write
+                status = 6;
+                continue;
+            }
+            const uint8_t* page = pools[tier] + phys * (int64_t)orc_page_bytes(tier);
+            orc_unpack_token(tier, (int)(t % ORC_PAGE), page, leaf, up, &r16, &s16, vq);
+            decode_key_one(ORC_D, leaf, up, r16, ORC_BLEAF[tier], ORC_BUP[tier], K + n * ORC_D, w);
+            orc_decode_values(1, ORC_D, vq, &s16, V + n * ORC_D);
+            ++n;
+        }
+        orc_attention(n, ORC_D, K, V, G, q + ((int64_t)b * H_q + (int64_t)g * G) * ORC_D,
+                      out + (int64_t)s * G * ORC_D, lse + (int64_t)s * G);
+        free(K);
+        free(V);
+    }
+    return status;
+}
+
+/* ---------------------------------------------------------------- RDR -- */
+
+/* Lagrangian tier choice for one unit: argmin over t of U*eps[t] + lambda*R[t],
+ * ties to the lower index (higher precision).  Index 0..3 = T1, T2, T3, drop. */
+static int rdr_choice(double U, const double* eps, const double* R, double lambda)
+{
+    int best = 0;
+    double bc = U * eps[0] + lambda * R[0];
+    for (int t = 1; t < 4; ++t) {
+        double c = U * eps[t] + lambda * R[t];
+        if (c < bc) { bc = c; best = t; }
+    }
+    return best;
+}
+
+/* Rate-distortion retention.  Units are (kv head g, sequence b, page p) for
+ * p < ceil(seq_len/16).  U = sum of the per-token utilities of the valid
+ * tokens (t = 0..15 in order).  Rate R = page bytes of the tier (drop = 0);
+ * distortion D = U * eps[tier].  The first n_sink and last n_recent pages of
+ * each sequence are forced to T1 and count against the budget.  The other
+ * units take argmin D + lambda R; lambda is found by doubling from 1 until the
+ * bytes fit, then 100 bisection steps, keeping the feasible end.
+ * utility: [H_kv][total_pages*16] (token slot of page i at i*16 + slot).
+ * tiers: [H_kv][total_pages], written 1..3 or 0 (drop) for pages that hold
+ * tokens; other entries are left untouched.
+ * Returns 0, or 3 when the forced pages alone exceed the budget. */
+int orc_rdr_assign(int B, int H_kv, int64_t total_pages, const int32_t* page_offsets,
+                   const int32_t* seq_lens, const float* utility, const double* eps,
+                   int64_t budget, int n_sink, int n_recent, uint8_t* tiers,
+                   double* lambda_out, int64_t* bytes_out)
+{
+    double R[4];
+    for (int t = 0; t < 3; ++t) R[t] = (double)orc_page_bytes(t + 1);
+    R[3] = 0.0;
+    /* flatten units */
+    int64_t n_units = 0;
+    for (int b = 0; b < B; ++b) n_units += (seq_lens[b] + ORC_PAGE - 1) / ORC_PAGE;
+    n_units *= H_kv;
+    double* U = (double*)malloc(sizeof(double) * (size_t)(n_units > 0 ? n_units : 1));
+    int64_t* idx = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n_units > 0 ? n_units : 1));
+    uint8_t* forced = (uint8_t*)malloc((size_t)(n_units > 0 ? n_units : 1));
+    int64_t u = 0, forced_bytes = 0;
+    for (int g = 0; g < H_kv; ++g)
+        for (int b = 0; b < B; ++b) {
+            int64_t len = seq_lens[b];
+            int64_t np = (len + ORC_PAGE - 1) / ORC_PAGE;
+            for (int64_t p = 0; p < np; ++p) {
+                int64_t e = (int64_t)g * total_pages + page_offsets[b] + p;
+                double s = 0.0;
+                for (int k = 0; k < ORC_PAGE && p * ORC_PAGE + k < len; ++k)
+                    s += (double)utility[e * ORC_PAGE + k];
+                U[u] = s;
+                idx[u] = e;
+                forced[u] = (p < n_sink || p >= np - n_recent) ? 1 : 0;
+                if (forced[u]) forced_bytes += (int64_t)R[0];
+                ++u;
+            }
+        }
+    if (forced_bytes > budget) {
+        free(U); free(idx); free(forced);
+        return 3;
+    }
+#define RDR_BYTES(lam, out_bytes)                                               \
+    do {                                                                        \
+        int64_t acc_ = 0;                                                       \
+        for (int64_t i_ = 0; i_ < n_units; ++i_)                                \
+            acc_ += forced[i_] ? (int64_t)R[0] : (int64_t)R[rdr_choice(U[i_], eps, R, (lam))]; \
+        (out_bytes) = acc_;                                                     \
+    } while (0)
+    double lo = 0.0, hi = 1.0;
+    int64_t bh;
+    RDR_BYTES(hi, bh);
+    for (int k = 0; k < 2000 && bh > budget; ++k) {
+        hi = hi * 2.0;
+        RDR_BYTES(hi, bh);
+    }
+    for (int it = 0; it < 100; ++it) {
+        double mid = lo + (hi - lo) / 2.0;
+        int64_t bm;
+        RDR_BYTES(mid, bm);
+        if (bm <= budget) hi = mid;
+        else lo = mid;
+    }
+    RDR_BYTES(hi, bh);
+#undef RDR_BYTES
+    for (int64_t i = 0; i < n_units; ++i) {
+        int t = forced[i] ? 0 : rdr_choice(U[i], eps, R, hi);
+        tiers[idx[i]] = (uint8_t)(t == 3 ? 0 : t + 1);
+    }
+    *lambda_out = hi;
+    *bytes_out = bh;
+    free(U); free(idx); free(forced);
+    return 0;
+}
+
+int orc_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

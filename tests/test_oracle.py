@@ -1,0 +1,480 @@
+"""Pins for the fp64 CPU oracle, checked against things other than itself:
+library routines (numpy's fp16 conversion), hand-worked cases, closed forms,
+explicit small-d formulas, rigorous error bounds and brute force.
+
+Each test names the fact it pins.  None of them needs a GPU.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+TIERS = oracle.TIER_BITS
+
+
+def _dir_err(d, b_leaf, b_up):
+    """Worst-case direction error: half a leaf step plus half an upper step per
+    upper level (levels act on disjoint subspaces of total weight 1)."""
+    levels = int(round(math.log2(d // 2)))
+    return math.pi / 2 ** b_leaf + levels * (math.pi / 2) / (2 * (2 ** b_up - 1))
+
+
+def _random_codes(rng, n, d, b_leaf, b_up, inner_only=False):
+    L = d // 2
+    leaf = rng.integers(0, 2 ** b_leaf, size=(n, L)).astype(np.uint8)
+    lo, hi = (1, 2 ** b_up - 2) if inner_only else (0, 2 ** b_up - 1)
+    up = rng.integers(lo, hi, size=(n, L - 1), endpoint=True).astype(np.uint8)
+    # radii: random normal fp16 values in [0.25, 64)
+    r = rng.uniform(0.25, 64.0, size=n)
+    r16 = r.astype(np.float16).view(np.uint16)
+    return leaf, up, r16
+
+
+# ------------------------------------------------------------------ fp16 --
+def test_fp16_rounding_matches_numpy():
+    """Pin: the oracle's double->half RNE equals numpy's conversion (a library
+    routine), on random values over the whole range, halfway ties, subnormals
+    and the overflow edge."""
+    rng = np.random.default_rng(1)
+    xs = list(rng.standard_normal(3000) * np.exp(rng.uniform(-25, 12, 3000)))
+    # exact ties between consecutive halves, subnormal ties and the overflow edge
+    h = np.arange(0, 0x7bff, 7, dtype=np.uint16).view(np.float16).astype(np.float64)
+    xs += list((h[:-1] + h[1:]) / 2)
+    xs += [0.0, -0.0, 65504.0, 65519.99, 65520.0, 1e9, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26,
+           2.0 ** -26, 6.1e-5, -6.1e-5, 1 / 127, 2 / 127]
+    for x in xs:
+        want = int(np.array(x, np.float64).astype(np.float16).view(np.uint16))
+        got = oracle.f64_to_f16_bits(x)
+        assert got == want, (x, hex(got), hex(want))
+    for bits in range(0, 0x10000, 3):
+        want = float(np.array(bits, np.uint16).view(np.float16))
+        got = oracle.f16_bits_to_f64(bits)
+        if math.isnan(want):
+            assert math.isnan(got)
+        else:
+            assert got == want
+
+
+# -------------------------------------------------------------- hand case --
+def test_hand_case():
+    """Pin: the two-token d = 4 case worked by hand (tests/golden/hand_case.json)."""
+    g = json.load(open(os.path.join(GOLD, "hand_case.json")))
+    K = np.array(g["K"], np.float64)
+    V = np.array(g["V"], np.float64)
+    q = np.array(g["q"], np.float64)
+    c = oracle.encode(K, V, bits=(8, 8, 8))
+    assert c["leaf"].tolist() == g["leaf_codes"]
+    assert c["up"].tolist() == g["up_codes"]
+    assert [oracle.f16_bits_to_f64(x) for x in c["r16"]] == g["r"]
+    assert [oracle.f16_bits_to_f64(x) for x in c["s16"]] == g["vscale"]
+    assert c["vq"].tolist() == g["vq"]
+    kh = oracle.decode_keys(c["leaf"], c["up"], c["r16"], 8, 8)
+    np.testing.assert_allclose(kh, K, atol=1e-15)
+    tl = oracle.tree_logits(c["leaf"], c["up"], c["r16"], 8, 8, q)
+    np.testing.assert_allclose(tl, g["logits"], atol=1e-15)
+    vh = oracle.decode_values(c["vq"], c["s16"])
+    out, lse = oracle.attention(kh, vh, q[None])
+    p1 = 1.0 / (1.0 + math.exp(0.5))
+    p2 = 1.0 / (1.0 + math.exp(-0.5))
+    s1, s2 = g["vscale"]
+    want_out = [p1 * 127 * s1, -p1 * 127 * s1, p2 * 127 * s2, 0.0]
+    want_lse = 1.0 + math.log(1.0 + math.exp(-0.5))
+    np.testing.assert_allclose(out[0], want_out, rtol=0, atol=1e-14)
+    assert abs(lse[0] - want_lse) < 1e-14
+    # and the numbers written out in decimal in the derivation
+    np.testing.assert_allclose(out[0], [0.3775176255444346, -0.3775176255444346,
+                                        1.2448426785986308, 0.0], atol=1e-14)
+    assert abs(lse[0] - 1.4740769841801067) < 1e-14
+
+
+# ---------------------------------------------------------- tree identity --
+@pytest.mark.parametrize("tier", [1, 2, 3])
+@pytest.mark.parametrize("d", [4, 8, 16, 64, 128])
+def test_tree_logit_equals_dense_dot(tier, d):
+    """Pin: the bottom-up angle-domain tree (leaf q.(cos, sin), node
+    cos psi S_L + sin psi S_R) equals q . decode(codes) / sqrt(d) to 1e-12,
+    for random codes of every tier (both are the same multilinear form)."""
+    b_leaf, b_up, _ = TIERS[tier]
+    rng = np.random.default_rng(10 * tier + d)
+    leaf, up, r16 = _random_codes(rng, 300, d, b_leaf, b_up)
+    for _ in range(3):
+        q = rng.standard_normal(d) * rng.uniform(0.1, 5)
+        tl = oracle.tree_logits(leaf, up, r16, b_leaf, b_up, q)
+        kh = oracle.decode_keys(leaf, up, r16, b_leaf, b_up)
+        dense = kh @ q / math.sqrt(d)
+        r = r16.view(np.float16).astype(np.float64)
+        scale = np.maximum(1.0, r * np.linalg.norm(q) / math.sqrt(d))
+        assert np.all(np.abs(tl - dense) <= 1e-12 * scale)
+
+
+def test_decode_matches_explicit_small_d():
+    """Pin: decode for d = 4 and d = 8 equals the recursive-polar direction
+    written out by hand as products of cosines and sines."""
+    rng = np.random.default_rng(3)
+    for tier, (bl, bu, _) in TIERS.items():
+        leaf, up, r16 = _random_codes(rng, 50, 4, bl, bu)
+        kh = oracle.decode_keys(leaf, up, r16, bl, bu)
+        for i in range(50):
+            f0 = 2 * math.pi * leaf[i, 0] / 2 ** bl
+            f1 = 2 * math.pi * leaf[i, 1] / 2 ** bl
+            ps = (math.pi / 2) * up[i, 0] / (2 ** bu - 1)
+            r = float(r16[i:i + 1].view(np.float16)[0])
+            want = r * np.array([math.cos(ps) * math.cos(f0), math.cos(ps) * math.sin(f0),
+                                 math.sin(ps) * math.cos(f1), math.sin(ps) * math.sin(f1)])
+            np.testing.assert_allclose(kh[i], want, atol=1e-13 * r)
+        leaf, up, r16 = _random_codes(rng, 50, 8, bl, bu)
+        kh = oracle.decode_keys(leaf, up, r16, bl, bu)
+        for i in range(50):
+            f = [2 * math.pi * leaf[i, j] / 2 ** bl for j in range(4)]
+            # level order: level-1 nodes (leaves 0,1) and (leaves 2,3), then the root
+            a, b, root = [(math.pi / 2) * up[i, m] / (2 ** bu - 1) for m in range(3)]
+            w = [math.cos(root) * math.cos(a), math.cos(root) * math.sin(a),
+                 math.sin(root) * math.cos(b), math.sin(root) * math.sin(b)]
+            r = float(r16[i:i + 1].view(np.float16)[0])
+            want = r * np.array([w[j // 2] * (math.cos(f[j // 2]) if j % 2 == 0 else math.sin(f[j // 2]))
+                                 for j in range(8)])
+            np.testing.assert_allclose(kh[i], want, atol=1e-13 * r)
+
+
+# ---------------------------------------------------------- encode checks --
+@pytest.mark.parametrize("tier", [1, 2, 3])
+def test_grid_points_reencode_exactly(tier):
+    """Pin: a key placed exactly on the angle grid (decode of random codes)
+    re-encodes to the same codes and radius."""
+    bl, bu, vb = TIERS[tier]
+    rng = np.random.default_rng(20 + tier)
+    leaf, up, r16 = _random_codes(rng, 400, 128, bl, bu, inner_only=True)
+    kh = oracle.decode_keys(leaf, up, r16, bl, bu)
+    c = oracle.encode(kh, np.zeros_like(kh), bits=(bl, bu, vb))
+    assert np.array_equal(c["leaf"], leaf)
+    assert np.array_equal(c["up"], up)
+    assert np.array_equal(c["r16"], r16)
+
+
+def test_zero_subtrees_and_axis_keys():
+    """Pin: with the end-inclusive upper grid a zero half of the key gives an
+    exact 0 or pi/2 upper angle, zero pairs get code 0, and axis keys decode
+    exactly."""
+    d = 16
+    K = np.zeros((4, d))
+    K[0, 0] = 3.0           # all weight in the leftmost leaf
+    K[1, d - 1] = -2.0      # all weight in the last coordinate
+    K[2, 4:8] = [1, 1, 1, 1]
+    K[3, :] = 0.0           # the zero key
+    c = oracle.encode(K, np.zeros_like(K), bits=(8, 8, 8))
+    assert c["up"][0].tolist() == [0] * 7
+    assert c["leaf"][0].tolist() == [0] * 8
+    assert c["up"][1].tolist() == [0, 0, 0, 255, 0, 255, 255]
+    assert c["leaf"][1].tolist() == [0] * 7 + [192]  # atan2(-2, 0) = -pi/2 -> -64 mod 256
+    assert c["up"][3].tolist() == [0] * 7 and c["leaf"][3].tolist() == [0] * 8
+    assert oracle.f16_bits_to_f64(c["r16"][3]) == 0.0
+    kh = oracle.decode_keys(c["leaf"], c["up"], c["r16"], 8, 8)
+    np.testing.assert_allclose(kh[0], K[0], atol=1e-15)
+    np.testing.assert_allclose(kh[1], K[1], atol=1e-15)
+    np.testing.assert_allclose(kh[3], 0.0)
+
+
+@pytest.mark.parametrize("tier", [1, 2, 3])
+def test_encode_error_bounds(tier):
+    """Pin: for every tier the decoded direction is within the worst-case
+    angle error bound of the true direction, |v - v_hat| <= s/2, and the radius
+    is the fp16 rounding of |k|."""
+    bl, bu, vb = TIERS[tier]
+    rng = np.random.default_rng(30 + tier)
+    sig = rng.lognormal(0, 0.5, 128)
+    sig[rng.choice(128, 4, replace=False)] *= 8
+    K = rng.standard_normal((2000, 128)) * sig
+    V = rng.standard_normal((2000, 128))
+    c = oracle.encode(K, V, tier)
+    kh = oracle.decode_keys(c["leaf"], c["up"], c["r16"], bl, bu)
+    r = np.linalg.norm(K, axis=1)
+    rh = c["r16"].view(np.float16).astype(np.float64)
+    assert np.all(np.abs(r - rh) <= np.abs(r) * 2.0 ** -11 + 1e-300)
+    u = K / r[:, None]
+    uh = kh / rh[:, None]
+    err = np.linalg.norm(u - uh, axis=1)
+    assert err.max() <= _dir_err(128, bl, bu) + 1e-12
+    vh = oracle.decode_values(c["vq"], c["s16"])
+    s = c["s16"].view(np.float16).astype(np.float64)
+    assert np.all(np.abs(V - vh) <= s[:, None] / 2 + 1e-15)
+    Q = 127 if vb == 8 else 7
+    assert np.abs(c["vq"]).max() <= Q
+
+
+@pytest.mark.parametrize("tier", [1, 2, 3])
+def test_logits_within_bound_of_dense(tier):
+    """Pin: every code-domain logit is within delta_t = |q| (r e_dir + |r - r_hat|)
+    / sqrt(d) of the exact dense logit q.k / sqrt(d); T1 attention stays within
+    the derived bounds of exact dense fp64 attention (|dlse| <= max delta,
+    |dout| <= (e^(2 max delta) - 1) max|v_hat| + max s / 2)."""
+    bl, bu, _ = TIERS[tier]
+    rng = np.random.default_rng(40 + tier)
+    d = 128
+    sig = rng.lognormal(0, 0.5, d)
+    K = rng.standard_normal((2048, d)) * sig
+    V = rng.standard_normal((2048, d))
+    q = rng.standard_normal((4, d))
+    c = oracle.encode(K, V, tier)
+    kh = oracle.decode_keys(c["leaf"], c["up"], c["r16"], bl, bu)
+    vh = oracle.decode_values(c["vq"], c["s16"])
+    r = np.linalg.norm(K, axis=1)
+    rh = c["r16"].view(np.float16).astype(np.float64)
+    e = _dir_err(d, bl, bu)
+    for h in range(4):
+        delta = np.linalg.norm(q[h]) * (r * e + np.abs(r - rh)) / math.sqrt(d)
+        l_ex = K @ q[h] / math.sqrt(d)
+        l_or = oracle.tree_logits(c["leaf"], c["up"], c["r16"], bl, bu, q[h])
+        assert np.all(np.abs(l_or - l_ex) <= delta + 1e-12)
+        eps_max = delta.max()
+        out_o, lse_o = oracle.attention(kh, vh, q[h:h + 1])
+        m = l_ex.max()
+        p = np.exp(l_ex - m)
+        out_d = (p[:, None] * V).sum(0) / p.sum()
+        lse_d = m + math.log(p.sum())
+        assert abs(lse_o[0] - lse_d) <= eps_max + 1e-12
+        s = c["s16"].view(np.float16).astype(np.float64)
+        bound = (math.exp(2 * eps_max) - 1) * np.abs(vh).max() + s.max() / 2
+        assert np.abs(out_o[0] - out_d).max() <= bound + 1e-12
+
+
+# -------------------------------------------------------------- attention --
+def _small_cache(rng, tiers_per_page, seq_len, H_kv=1, G=4):
+    """A one-sequence cache built with the oracle's own encoder and packer."""
+    n_pages = len(tiers_per_page)
+    tiers = np.array([tiers_per_page] * H_kv, np.uint8)
+    table = oracle.build_page_table(tiers)
+    K = rng.standard_normal((seq_len, H_kv, 128)) * rng.lognormal(0, 0.5, 128)
+    V = rng.standard_normal((seq_len, H_kv, 128))
+    counts = [int((tiers == t).sum()) for t in (1, 2, 3)]
+    pools = oracle.encode_cache(K, V, np.zeros(seq_len, np.int32), np.arange(seq_len),
+                                np.array([0, n_pages]), table, counts)
+    cache = dict(B=1, H_q=G * H_kv, H_kv=H_kv, page_offsets=np.array([0, n_pages], np.int32),
+                 seq_lens=np.array([seq_len], np.int32), page_table=table, pools=pools)
+    return cache, K, V
+
+
+def test_dropped_pages_contribute_exactly_zero():
+    """Pin: attention over a cache with dropped pages equals, bit for bit,
+    attention over the same tokens with the dropped tokens deleted."""
+    rng = np.random.default_rng(5)
+    tiers = [1, 0, 2, 3, 0, 0, 1, 2]
+    cache, K, V = _small_cache(rng, tiers, 8 * 16 - 5)
+    q = rng.standard_normal((1, 4, 128))
+    out, lse = oracle.cache_attention(cache, q, [(0, 0)])
+    keep_k, keep_v = [], []
+    for t in range(K.shape[0]):
+        tier = tiers[t // 16]
+        if tier == 0:
+            continue
+        c = oracle.encode(K[t:t + 1, 0], V[t:t + 1, 0], tier)
+        bl, bu, _ = TIERS[tier]
+        keep_k.append(oracle.decode_keys(c["leaf"], c["up"], c["r16"], bl, bu)[0])
+        keep_v.append(oracle.decode_values(c["vq"], c["s16"])[0])
+    out2, lse2 = oracle.attention(np.array(keep_k), np.array(keep_v), q[0])
+    assert np.array_equal(out[0], out2)
+    assert np.array_equal(lse[0], lse2)
+
+
+def test_special_cases():
+    """Pin: q = 0 gives the mean of the kept values and lse = ln(#kept); one
+    kept token gives its value and its logit; no kept token gives out = 0,
+    lse = -inf."""
+    rng = np.random.default_rng(6)
+    cache, K, V = _small_cache(rng, [2, 0, 3], 40)
+    q = np.zeros((1, 4, 128))
+    out, lse = oracle.cache_attention(cache, q, [(0, 0)])
+    kept = [t for t in range(40) if (t // 16) != 1]
+    vh = []
+    for t in kept:
+        tier = [2, 0, 3][t // 16]
+        c = oracle.encode(K[t:t + 1, 0], V[t:t + 1, 0], tier)
+        vh.append(oracle.decode_values(c["vq"], c["s16"])[0])
+    np.testing.assert_allclose(out[0, 0], np.mean(vh, 0), atol=1e-14)
+    assert abs(lse[0, 0] - math.log(len(kept))) < 1e-14
+
+    cache, K, V = _small_cache(rng, [1], 1)
+    q = rng.standard_normal((1, 4, 128))
+    out, lse = oracle.cache_attention(cache, q, [(0, 0)])
+    c = oracle.encode(K[:, 0], V[:, 0], 1)
+    vh = oracle.decode_values(c["vq"], c["s16"])[0]
+    for h in range(4):
+        np.testing.assert_allclose(out[0, h], vh, atol=1e-15)
+        lt = oracle.tree_logits(c["leaf"], c["up"], c["r16"], 8, 8, q[0, h])[0]
+        assert abs(lse[0, h] - lt) < 1e-12
+
+    cache, K, V = _small_cache(rng, [0, 0], 20)
+    out, lse = oracle.cache_attention(cache, q, [(0, 0)])
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+# ------------------------------------------------------------ page format --
+def test_page_layout_golden():
+    """Pin: packed bytes equal the hand-worked bytes in tests/golden/page_layout.json."""
+    g = json.load(open(os.path.join(GOLD, "page_layout.json")))
+    for t in (1, 2, 3):
+        assert oracle.page_bytes(t) == g["page_bytes"][str(t)]
+    z_up = np.zeros(63, np.uint8)
+    z_v = np.zeros(128, np.int8)
+    # T3 leaf row of codes j mod 8
+    page = np.zeros(oracle.page_bytes(3), np.uint8)
+    leaf = (np.arange(64) % 8).astype(np.uint8)
+    oracle.pack_token(3, 0, leaf, z_up, 0, 0, z_v, page)
+    assert page[64:67].tolist() == g["t3_leaf_codes_j_mod_8_first_bytes"]
+    # T2 upper row of codes m
+    page = np.zeros(oracle.page_bytes(2), np.uint8)
+    up = np.arange(63).astype(np.uint8)
+    oracle.pack_token(2, 0, np.zeros(64, np.uint8), up, 0, 0, z_v, page)
+    off_up = 64 + 16 * 32
+    assert page[off_up:off_up + 3].tolist() == g["t2_up_codes_m_first_bytes"]
+    assert page[off_up + 46:off_up + 48].tolist() == g["t2_up_codes_m_bytes_46_47"]
+    # int4 nibbles
+    for pair, want in g["int4_pairs"]:
+        if want is None:
+            continue
+        page = np.zeros(oracle.page_bytes(2), np.uint8)
+        vq = np.zeros(128, np.int8)
+        vq[0:2] = pair
+        oracle.pack_token(2, 0, np.zeros(64, np.uint8), z_up, 0, 0, vq, page)
+        off_v = 64 + 16 * 32 + 16 * 48
+        assert page[off_v] == want
+
+
+def test_pack_unpack_roundtrip_and_independent_bitstream():
+    """Pin: pack/unpack round-trips for every tier and slot, and each packed
+    row equals the same codes assembled as one Python integer (bit i*b of the
+    row holds code i), other slots untouched and pad bits zero."""
+    rng = np.random.default_rng(7)
+    for t, (bl, bu, vb) in TIERS.items():
+        page = np.zeros(oracle.page_bytes(t), np.uint8)
+        rows = []
+        for slot in rng.permutation(16):
+            leaf = rng.integers(0, 2 ** bl, 64).astype(np.uint8)
+            up = rng.integers(0, 2 ** bu, 63).astype(np.uint8)
+            Q = 127 if vb == 8 else 7
+            vq = rng.integers(-Q, Q, 128, endpoint=True).astype(np.int8)
+            r16, s16 = int(rng.integers(0, 0x7bff)), int(rng.integers(0, 0x7bff))
+            oracle.pack_token(t, int(slot), leaf, up, r16, s16, vq, page)
+            rows.append((int(slot), leaf, up, r16, s16, vq))
+        for slot, leaf, up, r16, s16, vq in rows:
+            u = oracle.unpack_token(t, slot, page)
+            assert np.array_equal(u["leaf"], leaf) and np.array_equal(u["up"], up)
+            assert u["r16"] == r16 and u["s16"] == s16 and np.array_equal(u["vq"], vq)
+            lrow = 64 * bl // 8
+            urow = (63 * bu + 127) // 128 * 16
+            vrow = 128 * vb // 8
+            big = sum(int(c) << (i * bl) for i, c in enumerate(leaf))
+            assert bytes(page[64 + slot * lrow: 64 + (slot + 1) * lrow]) == big.to_bytes(lrow, "little")
+            big = sum(int(c) << (i * bu) for i, c in enumerate(up))
+            o = 64 + 16 * lrow
+            assert bytes(page[o + slot * urow: o + (slot + 1) * urow]) == big.to_bytes(urow, "little")
+            big = sum((int(c) & (2 ** vb - 1)) << (i * vb) for i, c in enumerate(vq))
+            o = 64 + 16 * lrow + 16 * urow
+            assert bytes(page[o + slot * vrow: o + (slot + 1) * vrow]) == big.to_bytes(vrow, "little")
+            assert int(page[2 * slot]) | int(page[2 * slot + 1]) << 8 == r16
+            assert int(page[32 + 2 * slot]) | int(page[33 + 2 * slot]) << 8 == s16
+
+
+def test_page_table_entries():
+    """Pin: entry = tier << 30 | pool index; the k-th page of a tier in table
+    order gets perm[k]."""
+    tiers = np.array([[1, 0, 2, 1, 3, 2, 0, 1]], np.uint8)
+    t = oracle.build_page_table(tiers).view(np.uint32)
+    assert t.tolist() == [[(1 << 30) | 0, 0, (2 << 30) | 0, (1 << 30) | 1, (3 << 30) | 0,
+                           (2 << 30) | 1, 0, (1 << 30) | 2]]
+    p1 = np.array([2, 0, 1], np.int32)
+    t = oracle.build_page_table(tiers, (p1, None, None)).view(np.uint32)
+    assert [x & 0x3fffffff for x in t[0, [0, 3, 7]]] == [2, 0, 1]
+
+
+# -------------------------------------------------------------------- RDR --
+EPS = np.array([1.1e-4, 2.75e-2, 7.12e-2, 2.0])
+RATE = [4160, 2368, 1984, 0]
+
+
+def _rdr_small(U_pages, budget, n_sink=0, n_recent=0):
+    """Units = pages of one sequence with one token each carrying utility U."""
+    n = len(U_pages)
+    util = np.zeros((1, n * 16), np.float32)
+    util[0, ::16] = U_pages
+    lens = np.array([16 * (n - 1) + 1], np.int32)
+    return oracle.rdr_assign(np.array([0, n], np.int32), lens, util, EPS, budget, n_sink,
+                             n_recent, 1)
+
+
+def test_rdr_hand_case():
+    """Pin: worked by hand.  Units U = 100 and U = 1, budget 4160 + 2368.
+    The U = 1 unit leaves T1 for T2 at lambda = 1*(eps2 - eps1)/(4160 - 2368),
+    the U = 100 unit only at 100x that, so the answer is (T1, T2) with lambda
+    at the first breakpoint."""
+    util = np.zeros((1, 32), np.float32)
+    util[0, 0] = 100.0
+    util[0, 16] = 1.0
+    tiers, lam, nb = oracle.rdr_assign(np.array([0, 2], np.int32), np.array([17], np.int32),
+                                       util, EPS, 4160 + 2368, 0, 0, 1)
+    assert tiers[0].tolist() == [1, 2]
+    assert nb == 4160 + 2368
+    lam_star = (EPS[1] - EPS[0]) / (4160 - 2368)
+    assert abs(lam - lam_star) <= 1e-12 * lam_star
+
+
+def test_rdr_brute_force_optimality():
+    """Pin: brute force over all 4^n assignments (n <= 8): the Lagrangian
+    answer has the least total distortion among all assignments using no more
+    bytes, it fits the budget, and forced units are T1."""
+    rng = np.random.default_rng(8)
+    for trial in range(25):
+        n = int(rng.integers(2, 9))
+        U = rng.lognormal(0, 1.5, n).astype(np.float32)
+        n_sink = int(rng.integers(0, 2))
+        total = sum(4160 for _ in range(n))
+        budget = int(rng.integers(4160 * n_sink + 1, total + 1))
+        tiers, lam, nb = _rdr_small(U, budget, n_sink=n_sink)
+        t = tiers[0]
+        idx = [0 if x == 1 else 1 if x == 2 else 2 if x == 3 else 3 for x in t]
+        R = sum(RATE[i] for i in idx)
+        assert R == nb <= budget
+        assert all(x == 1 for x in t[:n_sink])
+        D = sum(float(U[u]) * EPS[i] for u, i in enumerate(idx))
+        best = math.inf
+        for combo in itertools.product(range(4), repeat=n):
+            if any(combo[u] != 0 for u in range(n_sink)):
+                continue
+            if sum(RATE[i] for i in combo) <= R:
+                best = min(best, sum(float(U[u]) * EPS[i] for u, i in enumerate(combo)))
+        assert D <= best * (1 + 1e-12) + 1e-300
+
+
+def test_rdr_budget_monotone_and_infeasible():
+    """Pin: more budget never costs distortion and never reduces bytes; a
+    budget below the forced pages raises."""
+    rng = np.random.default_rng(9)
+    U = rng.lognormal(0, 1, 40).astype(np.float32)
+    prev_b, prev_d = -1, math.inf
+    for budget in np.linspace(4160 * 3, 4160 * 40, 25).astype(np.int64):
+        tiers, lam, nb = _rdr_small(U, int(budget), n_sink=2, n_recent=1)
+        idx = [{1: 0, 2: 1, 3: 2, 0: 3}[int(x)] for x in tiers[0]]
+        D = sum(float(U[u]) * EPS[i] for u, i in enumerate(idx))
+        assert nb <= budget and nb >= prev_b * 0 and D <= prev_d * (1 + 1e-12)
+        prev_b, prev_d = nb, D
+    with pytest.raises(OverflowError):
+        _rdr_small(U, 4160 * 3 - 1, n_sink=2, n_recent=1)
+
+
+def test_rdr_ties_go_to_higher_precision():
+    """Pin: when several tiers cost exactly the same in fp64 (equal eps, and
+    lambda*R below half an ulp of U*eps), the tie goes to the lower tier index,
+    i.e. the higher precision.  A budget that fits every page at T1 drives
+    lambda down to ~2^-100, where that happens."""
+    util = np.zeros((1, 5 * 16), np.float32)
+    util[0, ::16] = 1.0
+    eps = np.array([0.5, 0.5, 0.5, 2.0])
+    tiers, lam, nb = oracle.rdr_assign(np.array([0, 5], np.int32), np.array([65], np.int32),
+                                       util, eps, 5 * 4160, 0, 0, 1)
+    assert lam < 1e-20
+    assert tiers[0].tolist() == [1] * 5 and nb == 5 * 4160
