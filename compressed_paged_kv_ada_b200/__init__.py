@@ -1,0 +1,20 @@
+"""Spherical KV angle-domain attention (ADA) decode over a paged,
+tier-homogeneous compressed KV cache, for NVIDIA B200 (sm_100a).
+
+The compute lives in libsphkv.so (hand-written CUDA, C ABI in
+include/sphkv.h); this package only binds it.  Build it with
+`python -m compressed_paged_kv_ada_b200.build`.
+"""
+from ._lib import (  # noqa: F401
+    SphkvError,
+    lib,
+    make_cache,
+    sphkv_build_page_table,
+    sphkv_decode_attention,
+    sphkv_decode_workspace_bytes,
+    sphkv_encode,
+    sphkv_page_bytes,
+    sphkv_rdr_assign,
+    sphkv_rdr_workspace_bytes,
+)
+from .cache import PagedCache  # noqa: F401

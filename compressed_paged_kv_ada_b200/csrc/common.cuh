@@ -1,0 +1,85 @@
+// common.cuh -- format constants and device helpers shared by the libsphkv
+// kernels (encode, RDR, page table, decode).  Nothing here is used by, or
+// uses, the CPU oracle.
+//
+// Page format (Spherical KV, arXiv 2605.18856, Abstract: "tier-homogeneous
+// pages with lightweight metadata and coalesced reads"; the byte layout is
+// this library's):
+//   r[16] fp16 | vscale[16] fp16 | leaf rows | upper rows | value rows
+// with leaf row = 64 codes x b_leaf bits, upper row = 63 codes x b_up bits
+// rounded up to 16 bytes, value row = 128 x v_bits bits.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sphkv.h"
+
+namespace sphkv {
+
+constexpr int kD = SPHKV_HEAD_DIM;      // 128
+constexpr int kP = SPHKV_PAGE_TOKENS;   // 16
+constexpr int kLeaves = kD / 2;         // 64
+constexpr int kUpper = kD / 2 - 1;      // 63
+
+struct TierFmt {
+    int b_leaf, b_up, v_bits;
+    int leaf_row, up_row, v_row;   // bytes per token row
+    int off_leaf, off_up, off_v;   // byte offsets inside the page
+    int page_bytes;
+};
+
+__host__ __device__ constexpr TierFmt make_fmt(int bl, int bu, int vb)
+{
+    return TierFmt{bl,
+                   bu,
+                   vb,
+                   kLeaves * bl / 8,
+                   (kUpper * bu + 127) / 128 * 16,
+                   kD * vb / 8,
+                   4 * kP,
+                   4 * kP + kP * (kLeaves * bl / 8),
+                   4 * kP + kP * (kLeaves * bl / 8) + kP * ((kUpper * bu + 127) / 128 * 16),
+                   4 * kP + kP * (kLeaves * bl / 8) + kP * ((kUpper * bu + 127) / 128 * 16) +
+                       kP * (kD * vb / 8)};
+}
+
+// Tier index 1..3 (0 = drop).
+template <int T>
+struct Tier;
+template <>
+struct Tier<1> { static constexpr TierFmt f = make_fmt(8, 8, 8); };
+template <>
+struct Tier<2> { static constexpr TierFmt f = make_fmt(4, 6, 4); };
+template <>
+struct Tier<3> { static constexpr TierFmt f = make_fmt(3, 4, 4); };
+
+static_assert(Tier<1>::f.page_bytes == 4160, "T1 page");
+static_assert(Tier<2>::f.page_bytes == 2368, "T2 page");
+static_assert(Tier<3>::f.page_bytes == 1984, "T3 page");
+static_assert(Tier<1>::f.page_bytes % 16 == 0 && Tier<2>::f.page_bytes % 16 == 0 &&
+                  Tier<3>::f.page_bytes % 16 == 0,
+              "pages must be 16-byte multiples for bulk copies");
+
+__host__ __device__ inline int page_bytes_of(int t)
+{
+    return t == 1 ? Tier<1>::f.page_bytes
+                  : t == 2 ? Tier<2>::f.page_bytes : t == 3 ? Tier<3>::f.page_bytes : 0;
+}
+
+// Page-table entry: bits 31..30 tier, 29..0 pool page.
+__host__ __device__ inline int entry_tier(int32_t e) { return (int)(((uint32_t)e) >> 30); }
+__host__ __device__ inline int64_t entry_page(int32_t e) { return (int64_t)(((uint32_t)e) & 0x3fffffffu); }
+
+// Record a device-side error: the largest code wins, so the result does not
+// depend on the order in which threads report.
+__device__ inline void report(int32_t* status, int code)
+{
+    if (status) atomicMax(status, code);
+}
+
+}  // namespace sphkv
+
+// Host-side error text (per thread), set by the entry points.
+void sphkv_set_error(const char* fmt, ...);

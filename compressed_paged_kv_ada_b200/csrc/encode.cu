@@ -1,0 +1,252 @@
+// encode.cu -- dense K/V rows -> tier pages (prefill and append).
+//
+// Spherical KV (arXiv 2605.18856), Abstract: ADA stores each key "in a
+// spherical parameterization consisting of a scalar radius and compact angle
+// codes".  The recursive-polar tree, grids and bit layout are this library's
+// fixed format (see include/sphkv.h).
+//
+// One warp per (token, kv head).  Lane l owns dims 4l..4l+3, i.e. leaves 2l and
+// 2l+1 and the level-1 node l; higher tree levels combine partial sums of
+// squares with shuffles.  All angle math is fp64 with explicit _rn intrinsics
+// and the file is compiled with -fmad=false, so no product is fused into an
+// add and the codes match a plain fp64 reference bit for bit.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace sphkv {
+namespace {
+
+constexpr double kPi = 3.141592653589793;     // the double nearest pi
+constexpr double kPi2 = 1.5707963267948966;   // pi / 2 (exact half of kPi)
+constexpr int kEncWarps = 8;
+
+struct EncParams {
+    const void* K;
+    const void* V;
+    int dtype;
+    const int32_t* tok_seq;
+    const int32_t* tok_pos;
+    int64_t n_tok;
+    int B, H_kv;
+    int64_t total_pages;
+    const int32_t* page_offsets;
+    const int32_t* page_table;
+    uint8_t* pool[4];
+    int64_t pool_pages[4];
+    int32_t* status;
+};
+
+__device__ inline double load_elem(const void* base, int64_t idx, int dtype)
+{
+    if (dtype == SPHKV_DTYPE_BF16) {
+        const __nv_bfloat16* p = (const __nv_bfloat16*)base;
+        return (double)__bfloat162float(p[idx]);
+    }
+    return (double)((const float*)base)[idx];
+}
+
+// Leaf code: phi = atan2(y, x) on the periodic grid c * 2pi / 2^b.
+__device__ inline int leaf_code(double x, double y, int b)
+{
+    if (x == 0.0 && y == 0.0) return 0;
+    double phi = atan2(y, x);
+    double t = rint(__ddiv_rn(__dmul_rn(phi, (double)(1 << b)), 2.0 * kPi));
+    long long M = 1LL << b;
+    long long c = (long long)t;
+    c = ((c % M) + M) % M;
+    return (int)c;
+}
+
+// Upper code: psi = atan2(|R|, |L|) on the end-inclusive grid c*(pi/2)/(2^b-1).
+__device__ inline int upper_code(double ss_l, double ss_r, int b)
+{
+    double top = (double)((1 << b) - 1);
+    double nl = sqrt(ss_l), nr = sqrt(ss_r);
+    double psi = (nl == 0.0 && nr == 0.0) ? 0.0 : atan2(nr, nl);
+    double t = rint(__ddiv_rn(__dmul_rn(psi, top), kPi2));
+    t = fmin(fmax(t, 0.0), top);
+    return (int)t;
+}
+
+// 32-bit word w of a bit stream of n codes of b bits each, LSB first.
+__device__ inline uint32_t stream_word(const uint8_t* codes, int n, int b, int w)
+{
+    uint32_t word = 0;
+    int first = (32 * w) / b;
+    int last = (32 * w + 31) / b;
+    if (last > n - 1) last = n - 1;
+    for (int i = first; i <= last; ++i) {
+        int sh = i * b - 32 * w;
+        uint64_t c = codes[i];
+        word |= sh >= 0 ? (uint32_t)(c << sh) : (uint32_t)(c >> (-sh));
+    }
+    return word;
+}
+
+template <int T>
+__device__ void encode_token(const EncParams& p, int64_t i, int g, uint8_t* page, int slot,
+                             uint8_t* sleaf, uint8_t* sup, int lane)
+{
+    constexpr TierFmt F = Tier<T>::f;
+    const unsigned full = 0xffffffffu;
+    int64_t row = (i * p.H_kv + g) * kD + 4 * lane;
+    double k[4], v[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        k[c] = __dadd_rn(load_elem(p.K, row + c, p.dtype), 0.0);   // -0 -> +0
+        v[c] = load_elem(p.V, row + c, p.dtype);
+    }
+    // leaves 2l, 2l+1 and level-1 node l
+    double ssa = __dadd_rn(__dmul_rn(k[0], k[0]), __dmul_rn(k[1], k[1]));
+    double ssb = __dadd_rn(__dmul_rn(k[2], k[2]), __dmul_rn(k[3], k[3]));
+    sleaf[2 * lane] = (uint8_t)leaf_code(k[0], k[1], F.b_leaf);
+    sleaf[2 * lane + 1] = (uint8_t)leaf_code(k[2], k[3], F.b_leaf);
+    sup[lane] = (uint8_t)upper_code(ssa, ssb, F.b_up);
+    double ss = __dadd_rn(ssa, ssb);
+    // levels 2..6: node m of level l sits at lane m << (l-1)
+    int base = 32;
+#pragma unroll
+    for (int lvl = 1, width = 16; lvl <= 5; ++lvl, width >>= 1) {
+        double ssr = __shfl_down_sync(full, ss, 1 << (lvl - 1));
+        if ((lane & ((2 << (lvl - 1)) - 1)) == 0) {
+            int m = lane >> lvl;
+            sup[base + m] = (uint8_t)upper_code(ss, ssr, F.b_up);
+            ss = __dadd_rn(ss, ssr);
+        }
+        base += width;
+    }
+    // value scale: max |v| over the 128 channels
+    double a = fmax(fmax(fabs(v[0]), fabs(v[1])), fmax(fabs(v[2]), fabs(v[3])));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) a = fmax(a, __shfl_xor_sync(full, a, o));
+    const double Q = F.v_bits == 8 ? 127.0 : 7.0;
+    __half s16 = __double2half(__ddiv_rn(a, Q));
+    double s = (double)__half2float(s16);
+    int q[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        double t = s == 0.0 ? 0.0 : rint(__ddiv_rn(v[c], s));
+        q[c] = (int)fmin(fmax(t, -Q), Q);
+    }
+    __syncwarp();
+    // rows
+    uint8_t* lrow = page + F.off_leaf + slot * F.leaf_row;
+    uint8_t* urow = page + F.off_up + slot * F.up_row;
+    uint8_t* vrow = page + F.off_v + slot * F.v_row;
+    if (lane < F.leaf_row / 4)
+        ((uint32_t*)lrow)[lane] = stream_word(sleaf, kLeaves, F.b_leaf, lane);
+    if (lane < F.up_row / 4)
+        ((uint32_t*)urow)[lane] = stream_word(sup, kUpper, F.b_up, lane);
+    if (F.v_bits == 8) {
+        uint32_t w = (uint32_t)(q[0] & 0xff) | ((uint32_t)(q[1] & 0xff) << 8) |
+                     ((uint32_t)(q[2] & 0xff) << 16) | ((uint32_t)(q[3] & 0xff) << 24);
+        ((uint32_t*)vrow)[lane] = w;
+    } else {
+        uint16_t w = (uint16_t)((q[0] & 0xf) | ((q[1] & 0xf) << 4) | ((q[2] & 0xf) << 8) |
+                                ((q[3] & 0xf) << 12));
+        ((uint16_t*)vrow)[lane] = w;
+    }
+    if (lane == 0) {
+        __half r16 = __double2half(sqrt(ss));
+        ((__half*)page)[slot] = r16;
+        ((__half*)(page + 2 * kP))[slot] = s16;
+        if (__hisinf(r16) || __hisinf(s16)) report(p.status, SPHKV_ERR_RANGE);
+    }
+}
+
+__global__ void __launch_bounds__(kEncWarps * 32) encode_kernel(EncParams p)
+{
+    __shared__ uint8_t s_leaf[kEncWarps][kLeaves];
+    __shared__ uint8_t s_up[kEncWarps][kUpper + 1];
+    int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    int64_t wg = (int64_t)blockIdx.x * kEncWarps + wib;
+    if (wg >= p.n_tok * p.H_kv) return;
+    int64_t i = wg / p.H_kv;
+    int g = (int)(wg % p.H_kv);
+    int seq = p.tok_seq[i], pos = p.tok_pos[i];
+    if (seq < 0 || seq >= p.B || pos < 0) {
+        if (lane == 0) report(p.status, SPHKV_ERR_DATA);
+        return;
+    }
+    int64_t first = p.page_offsets[seq], cap = p.page_offsets[seq + 1] - first;
+    if (first < 0 || (int64_t)(pos / kP) >= cap || first + pos / kP >= p.total_pages) {
+        if (lane == 0) report(p.status, SPHKV_ERR_DATA);
+        return;
+    }
+    int32_t e = p.page_table[(int64_t)g * p.total_pages + first + pos / kP];
+    int t = entry_tier(e);
+    if (t == 0) return;
+    int64_t phys = entry_page(e);
+    if (phys >= p.pool_pages[t]) {
+        if (lane == 0) report(p.status, SPHKV_ERR_DATA);
+        return;
+    }
+    uint8_t* page = p.pool[t] + phys * (int64_t)page_bytes_of(t);
+    int slot = pos % kP;
+    if (t == 1) encode_token<1>(p, i, g, page, slot, s_leaf[wib], s_up[wib], lane);
+    else if (t == 2) encode_token<2>(p, i, g, page, slot, s_leaf[wib], s_up[wib], lane);
+    else encode_token<3>(p, i, g, page, slot, s_leaf[wib], s_up[wib], lane);
+}
+
+}  // namespace
+}  // namespace sphkv
+
+using namespace sphkv;
+
+extern "C" sphkv_status sphkv_encode(const sphkv_cache* c, const void* K, const void* V, int dtype,
+                                     const int32_t* tok_seq, const int32_t* tok_pos, int64_t n_tok,
+                                     int32_t* status_dev, void* stream)
+{
+    if (!c || (n_tok > 0 && (!K || !V || !tok_seq || !tok_pos))) {
+        sphkv_set_error("sphkv_encode: null argument");
+        return SPHKV_ERR_ARG;
+    }
+    if (dtype != SPHKV_DTYPE_F32 && dtype != SPHKV_DTYPE_BF16) {
+        sphkv_set_error("sphkv_encode: dtype must be SPHKV_DTYPE_F32 or SPHKV_DTYPE_BF16");
+        return SPHKV_ERR_ARG;
+    }
+    if (c->B <= 0 || c->H_kv <= 0 || c->total_pages < 0 || !c->page_offsets || !c->page_table) {
+        sphkv_set_error("sphkv_encode: bad cache descriptor");
+        return SPHKV_ERR_ARG;
+    }
+    if (n_tok < 0) {
+        sphkv_set_error("sphkv_encode: n_tok < 0");
+        return SPHKV_ERR_ARG;
+    }
+    if (n_tok == 0) return SPHKV_OK;
+    EncParams p{};
+    p.K = K;
+    p.V = V;
+    p.dtype = dtype;
+    p.tok_seq = tok_seq;
+    p.tok_pos = tok_pos;
+    p.n_tok = n_tok;
+    p.B = c->B;
+    p.H_kv = c->H_kv;
+    p.total_pages = c->total_pages;
+    p.page_offsets = c->page_offsets;
+    p.page_table = c->page_table;
+    for (int t = 1; t <= 3; ++t) {
+        p.pool[t] = c->pool[t - 1];
+        p.pool_pages[t] = c->pool[t - 1] ? c->pool_pages[t - 1] : 0;
+        if (c->pool[t - 1] && ((uintptr_t)c->pool[t - 1] & 15)) {
+            sphkv_set_error("sphkv_encode: pool %d is not 16-byte aligned", t);
+            return SPHKV_ERR_ARG;
+        }
+    }
+    p.status = status_dev;
+    int64_t warps = n_tok * c->H_kv;
+    int64_t blocks = (warps + kEncWarps - 1) / kEncWarps;
+    if (blocks > 0x7fffffffLL) {
+        sphkv_set_error("sphkv_encode: too many rows");
+        return SPHKV_ERR_ARG;
+    }
+    encode_kernel<<<(unsigned)blocks, kEncWarps * 32, 0, (cudaStream_t)stream>>>(p);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) {
+        sphkv_set_error("sphkv_encode: launch failed: %s", cudaGetErrorString(err));
+        return SPHKV_ERR_DEVICE;
+    }
+    return SPHKV_OK;
+}

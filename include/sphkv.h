@@ -1,0 +1,191 @@
+/*
+ * sphkv.h -- C ABI of libsphkv: Spherical KV angle-domain attention (ADA)
+ * decode over a paged, tier-homogeneous compressed KV cache, on NVIDIA B200
+ * (sm_100a).
+ *
+ * Method: "SPHERICAL KV: Angle-Domain Attention and Rate-Distortion Retention
+ * for Efficient Long-Context Inference" (arXiv 2605.18856), Abstract and AI
+ * Summary.  ADA stores each key as a scalar radius plus compact angle codes and
+ * computes attention logits directly from those codes, with no dense key
+ * rebuilt; RDR chooses keep/drop and a precision tier per unit under a fixed
+ * byte budget, so that pages are tier-homogeneous and read with coalesced
+ * loads.  The pages fix no bit layout; this library fixes the one below.
+ *
+ * Conventions for every entry point
+ *  - All array arguments are DEVICE pointers unless marked "host".  The caller
+ *    allocates and owns every buffer; the library allocates nothing.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously; nothing synchronises the host.
+ *  - The return value reports host-side argument errors and launch failures.
+ *    Problems only the device can see (bad page ids, fp16 overflow, a wait
+ *    that ran out) are written to `status_dev` (one device int32, may be NULL):
+ *    the kernels store the largest error code seen with an atomic max, so the
+ *    caller zeroes it first and reads it after synchronising.
+ *  - Head size d is 128 and pages hold 16 tokens.
+ *
+ * Format
+ *  Key k (d = 128) -> radius r = |k| rounded to fp16 (RNE), and the unit
+ *  direction in recursive-polar coordinates over a perfect binary tree:
+ *   - 64 leaf angles  phi_j = atan2(k[2j+1], k[2j])  (zero pair -> 0), coded on
+ *     a periodic grid of 2^b_leaf points c * 2pi / 2^b_leaf;
+ *   - 63 upper angles psi = atan2(|right half|, |left half|) in [0, pi/2],
+ *     coded on an end-inclusive grid c * (pi/2) / (2^b_up - 1);
+ *  rounding to nearest, ties to even, computed in fp64.  Upper nodes are in
+ *  level order: level 1 (parents of leaves 2m, 2m+1, m = 0..31), then level 2
+ *  (m = 0..15), ..., the root last.
+ *  The logit of query q is  r * S_root / sqrt(d), where a leaf gives
+ *  S = q[2j] cos(phi) + q[2j+1] sin(phi) and an upper node
+ *  S = cos(psi) S_left + sin(psi) S_right.
+ *  Value v -> per-token scale s = fp16(max|v| / Q) and codes
+ *  clamp(rint(v / s), -Q, Q), Q = 127 (int8) or 7 (int4); s = 0 gives 0 codes.
+ *
+ *  Tiers: T1 (b_leaf 8, b_up 8, int8 V, 4160 B/page), T2 (4, 6, int4, 2368 B),
+ *  T3 (3, 4, int4, 1984 B), or drop (no storage, excluded from the softmax).
+ *  Page of tier t (16-byte aligned fields, in this order):
+ *    r[16] fp16 | vscale[16] fp16 | leaf rows [16][8*b_leaf]
+ *    | upper rows [16][round_up_16(63*b_up/8)] | value rows [16][16*v_bits]
+ *  Codes are packed LSB-first into one little-endian bit stream per token row
+ *  (code i at bit i*b); int4 values put channel 2i in the low nibble (two's
+ *  complement).  Pad bits are 0.  Slots of tokens never written keep whatever
+ *  the caller put there (zero the pools to compare pages byte for byte).
+ *
+ *  Page table: int32 [H_kv][total_pages].  Bits 31..30 = tier (0 drop, 1..3),
+ *  bits 29..0 = page index inside that tier's pool.  Sequence b owns logical
+ *  pages page_offsets[b] .. page_offsets[b+1]-1 (for every kv head); token
+ *  position p lives in logical page p / 16, slot p % 16.  Query head h reads
+ *  kv head h / (H_q / H_kv).
+ */
+#ifndef SPHKV_H
+#define SPHKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int sphkv_status;
+#define SPHKV_OK 0
+#define SPHKV_ERR_ARG 1      /* null/misaligned pointer, bad size or shape */
+#define SPHKV_ERR_RANGE 2    /* radius or value scale overflows fp16; context > capacity */
+#define SPHKV_ERR_BUDGET 3   /* RDR: the forced pages alone exceed the budget */
+#define SPHKV_ERR_DEVICE 4   /* a CUDA call or launch failed */
+#define SPHKV_ERR_TIMEOUT 5  /* a bounded device-side wait ran out */
+#define SPHKV_ERR_DATA 6     /* device saw a page id outside its pool, a bad tier or position */
+
+#define SPHKV_PAGE_TOKENS 16
+#define SPHKV_HEAD_DIM 128
+
+#define SPHKV_DTYPE_F32 0
+#define SPHKV_DTYPE_BF16 1
+
+/* The paged cache.  A plain descriptor: every pointer is device memory owned
+ * by the caller; the struct itself lives on the host and is read only during
+ * the call that receives it. */
+typedef struct sphkv_cache {
+    int32_t B;                   /* sequences */
+    int32_t H_kv;                /* kv heads */
+    int64_t total_pages;         /* logical pages per kv head = page_offsets[B] */
+    const int32_t* page_offsets; /* [B+1], non-decreasing, page_offsets[0] = 0 */
+    const int32_t* seq_lens;     /* [B] tokens present; <= 16 * pages owned */
+    int32_t* page_table;         /* [H_kv][total_pages] entries, format above */
+    uint8_t* pool[3];            /* pools of T1, T2, T3 pages, 16-byte aligned */
+    int64_t pool_pages[3];       /* capacity of each pool in pages */
+} sphkv_cache;
+
+/* Bytes of one page of tier t (1..3); 0 for anything else. */
+int sphkv_page_bytes(int tier);
+
+/* Message of the last host-side error of the calling thread ("" if none). */
+const char* sphkv_last_error(void);
+
+/*
+ * sphkv_encode -- dense K/V rows -> tier pages (prefill and append).
+ *   Spherical KV Abstract (ADA: "a scalar radius and compact angle codes").
+ *   K, V: [n_tok][H_kv][128], dtype SPHKV_DTYPE_BF16 or SPHKV_DTYPE_F32.
+ *   tok_seq, tok_pos: [n_tok] int32, sequence and position of each row.
+ *   For each row and kv head the page-table entry of (seq, pos / 16) picks the
+ *   tier and pool page; the token is written to slot pos % 16 of that page.
+ *   Dropped pages are skipped.  Append is the same call with one row per
+ *   sequence.  Codes are computed in fp64 with no fused multiply-add, so they
+ *   match a plain fp64 reference bit for bit (short of libm atan2 differing in
+ *   the last ulp at an exact rounding boundary).
+ *   status_dev gets SPHKV_ERR_DATA for an out-of-range seq/pos/pool page
+ *   (the row is skipped) and SPHKV_ERR_RANGE for an fp16 overflow.
+ */
+sphkv_status sphkv_encode(const sphkv_cache* cache, const void* K, const void* V, int dtype,
+                          const int32_t* tok_seq, const int32_t* tok_pos, int64_t n_tok,
+                          int32_t* status_dev, void* stream);
+
+/*
+ * sphkv_rdr_workspace_bytes / sphkv_rdr_assign -- rate-distortion retention.
+ *   Spherical KV Abstract (RDR: keep/drop and precision tiers "under a fixed
+ *   budget", "a rate-distortion problem"); the Lagrangian form is this
+ *   library's reading.  Units are (kv head g, sequence b, page p) for
+ *   p < ceil(seq_len[b] / 16).  Page utility U = sum of `utility` over the
+ *   page's present tokens, summed in slot order in fp64.  Rate R = page bytes
+ *   of the tier (drop 0), distortion D = U * eps[tier].  The first n_sink and
+ *   last n_recent pages of each sequence are forced to T1 and count against the
+ *   budget.  Every other unit takes argmin_t U*eps[t] + lambda*R[t] (fp64, no
+ *   FMA, ties to the higher precision); lambda starts at 1, doubles until the
+ *   bytes fit (at most 2000 times), then 100 bisection steps keep the feasible
+ *   end.  The whole search runs on the device in one cooperative kernel.
+ *   utility: [H_kv][total_pages * 16] float (slot s of logical page i at
+ *            i * 16 + s).
+ *   eps: host [4] distortion per unit utility of T1, T2, T3, drop.
+ *   tiers_out: [H_kv][total_pages] uint8, written 1..3 (0 = drop) for pages
+ *            that hold tokens; other entries untouched.
+ *   lambda_out: device double; bytes_out: device int64 (total bytes chosen).
+ *   status_dev gets SPHKV_ERR_BUDGET when the forced pages exceed the budget
+ *   (tiers_out is then left untouched).
+ *   workspace: device, at least sphkv_rdr_workspace_bytes(...) bytes.
+ */
+size_t sphkv_rdr_workspace_bytes(int32_t B, int32_t H_kv, int64_t total_pages);
+sphkv_status sphkv_rdr_assign(const sphkv_cache* cache, const float* utility, const double* eps,
+                              int64_t budget_bytes, int32_t n_sink, int32_t n_recent,
+                              uint8_t* tiers_out, double* lambda_out, int64_t* bytes_out,
+                              void* workspace, size_t ws_bytes, int32_t* status_dev,
+                              void* stream);
+
+/*
+ * sphkv_build_page_table -- tiers -> page-table entries.
+ *   Spherical KV Abstract ("tier-homogeneous pages with lightweight
+ *   metadata").  tiers: [n_entries] uint8 (0 drop, 1..3) in table order; the
+ *   k-th entry of tier t (in table order) gets pool page perm_t[k], or k when
+ *   perm_t is NULL.  table: [n_entries] int32 out.  counts_out: device int64[3]
+ *   pages used per tier (may be NULL).  One kernel, a block-wide scan.
+ *   status_dev gets SPHKV_ERR_DATA if a tier value is above 3.
+ */
+sphkv_status sphkv_build_page_table(const uint8_t* tiers, int64_t n_entries, const int32_t* perm1,
+                                    const int32_t* perm2, const int32_t* perm3, int32_t* table,
+                                    int64_t* counts_out, int32_t* status_dev, void* stream);
+
+/*
+ * sphkv_decode_workspace_bytes / sphkv_decode_attention -- ADA decode.
+ *   Spherical KV Abstract ("computes attention logits directly from these
+ *   codes without reconstructing dense keys"; "a paged, block-local,
+ *   fusion-friendly decode path").  One decode query per sequence.
+ *   q: [B][H_q][128] fp32.  out: [B][H_q][128] fp32 = softmax-weighted sum of
+ *   the dequantised values of the kept tokens (t < seq_len, page not dropped);
+ *   lse: [B][H_q] fp32, natural-log log-sum-exp of the logits (scale 1/sqrt(d)
+ *   included).  A head with no kept token gets out = 0, lse = -inf.
+ *   H_q / H_kv must be 4.  Long contexts are split across SMs and the partial
+ *   (max, sum, out) triples merged with a log-sum-exp combine; the split
+ *   depends only on the shapes and the SM count, so results are reproducible
+ *   bit for bit and independent of the pool page ids.
+ *   workspace: device, 256-byte aligned, at least
+ *   sphkv_decode_workspace_bytes(B, H_q, H_kv, total_pages, n_sm) bytes, where
+ *   n_sm = 0 means the current device's SM count.
+ */
+size_t sphkv_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int64_t total_pages,
+                                    int32_t n_sm);
+sphkv_status sphkv_decode_attention(const sphkv_cache* cache, int32_t H_q, const float* q,
+                                    float* out, float* lse, void* workspace, size_t ws_bytes,
+                                    int32_t* status_dev, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPHKV_H */

@@ -66,6 +66,8 @@ def lib():
         L.orc_pack_token.argtypes = [c.c_int, c.c_int, P, P, c.c_uint16, c.c_uint16, P, P]
         L.orc_unpack_token.restype = None
         L.orc_unpack_token.argtypes = [c.c_int, c.c_int, P, P, P, P, P, P]
+        L.orc_pack_tokens.restype = None
+        L.orc_pack_tokens.argtypes = [c.c_int64, c.c_int, P, P, P, P, P, P, P, P]
         L.orc_build_page_table.restype = None
         L.orc_build_page_table.argtypes = [c.c_int64, P, P, P, P, P]
         L.orc_cache_attention.restype = c.c_int
@@ -274,9 +276,9 @@ def encode_cache(K, V, tok_seq, tok_pos, page_offsets, page_table, pool_pages):
             codes = encode(K[idx, g, :], V[idx, g, :], t)
             if codes["n_overflow"]:
                 raise OverflowError("radius or value scale overflows fp16")
-            pool = pools[t - 1]
-            for i, k in enumerate(idx):
-                lib().orc_pack_token(t, int(slot[k]), _p(codes["leaf"][i]), _p(codes["up"][i]),
-                                     int(codes["r16"][i]), int(codes["s16"][i]),
-                                     _p(codes["vq"][i]), _p(pool[phys[k]]))
+            dst = _c(phys[idx], np.int64)
+            sl = _c(slot[idx], np.int32)
+            lib().orc_pack_tokens(idx.size, t, _p(dst), _p(sl), _p(codes["leaf"]), _p(codes["up"]),
+                                  _p(codes["r16"]), _p(codes["s16"]), _p(codes["vq"]),
+                                  _p(pools[t - 1]))
     return pools

@@ -386,6 +386,19 @@ void orc_unpack_token(int t, int slot, const uint8_t* page, uint8_t* leaf, uint8
     }
 }
 
+/* Bulk form of orc_pack_token: token i goes to page dst_page[i] of `pool`
+ * (pages of tier t, orc_page_bytes(t) each), slot slot[i].  Codes are the
+ * [n][64], [n][63], [n], [n], [n][128] arrays of orc_encode_tokens. */
+void orc_pack_tokens(int64_t n, int t, const int64_t* dst_page, const int32_t* slot,
+                     const uint8_t* leaf, const uint8_t* up, const uint16_t* r16,
+                     const uint16_t* s16, const int8_t* vq, uint8_t* pool)
+{
+    int64_t pb = orc_page_bytes(t);
+    for (int64_t i = 0; i < n; ++i)
+        orc_pack_token(t, slot[i], leaf + i * (ORC_D / 2), up + i * (ORC_D / 2 - 1), r16[i], s16[i],
+                       vq + i * ORC_D, pool + dst_page[i] * pb);
+}
+
 /* Page-table entry: bits 31..30 tier (0 drop, 1 T1, 2 T2, 3 T3), bits 29..0
  * the page's index in that tier's pool. */
 void orc_build_page_table(int64_t n_entries, const uint8_t* tiers, const int32_t* perm1,
