@@ -65,6 +65,39 @@ def aggregate(times_ms, units, world):
     return sum(units) / (t / 1e3), t
 
 
+def reduce_over_ranks(ms_step: float, units: float, dist, device):
+    """Max of the per-rank step times and sum of the per-rank units, over all
+    ranks of the default process group (every rank calls this once)."""
+    import torch
+
+    tt = torch.tensor([ms_step], dtype=torch.float64, device=device)
+    uu = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    dist.all_reduce(uu, op=dist.ReduceOp.SUM)
+    return float(tt.item()), float(uu.item())
+
+
+def profiled_traffic(kernel_src: str, summary: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    kernel source has changed since the counters were taken."""
+    import hashlib
+
+    if not (os.path.exists(kernel_src) and os.path.exists(summary)):
+        return None
+    digest = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()[:16]
+    fields = {}
+    for line in open(summary):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    if fields.get("decode.cu sha256 prefix") != digest:
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def algorithmic_bytes(w) -> int:
     """Exact bytes the decode must move for one step: the bits of every kept
     token, one page-table entry per token-holding page, q, out and lse."""
@@ -297,11 +330,8 @@ def run_gpu(args):
     t_all = [ms_step]
     u_all = [units]
     if world > 1:
-        tt = torch.tensor([ms_step], dtype=torch.float64, device=dev)
-        uu = torch.tensor([units], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        dist.all_reduce(uu, op=dist.ReduceOp.SUM)
-        t_all, u_all = [float(tt.item())], [float(uu.item())]
+        t_max_r, u_sum = reduce_over_ranks(ms_step, units, dist, dev)
+        t_all, u_all = [t_max_r], [u_sum]
     value, t_max = aggregate(t_all, u_all, world)
 
     # ---- end to end through host buffers: q from pinned host memory in,
@@ -323,9 +353,7 @@ def run_gpu(args):
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+        e2e_ms, _ = reduce_over_ranks(e2e_ms, 0.0, dist, dev)
     e2e_value = sum(u_all) / (e2e_ms / 1e3)
 
     line = None
@@ -333,10 +361,8 @@ def run_gpu(args):
         algo = algorithmic_bytes(w)
         peak, peak_kind = measured_peaks()
         achieved = algo / (call_ms / 1e3) / 1e9
-        traffic = None
-        tpath = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
-        if os.path.exists(tpath):
-            traffic = json.load(open(tpath)).get("traffic_bytes_per_launch")
+        traffic = profiled_traffic(os.path.join(ROOT, "compressed_paged_kv_ada_b200", "csrc", "decode.cu"),
+                                   os.path.join(ROOT, "profiles", "decode_kernel_llama32k.md"))
         cb = cpu_baseline(w, q_np, budget_s=args.cpu_seconds) if (world == 1 and args.cpu_seconds > 0) else None
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

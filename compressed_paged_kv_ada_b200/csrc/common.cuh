@@ -4,10 +4,9 @@
 //
 // Page format (Spherical KV, arXiv 2605.18856, Abstract: "tier-homogeneous
 // pages with lightweight metadata and coalesced reads"; the byte layout is
-// this library's):
-//   r[16] fp16 | vscale[16] fp16 | leaf rows | upper rows | value rows
-// with leaf row = 64 codes x b_leaf bits, upper row = 63 codes x b_up bits
-// rounded up to 16 bytes, value row = 128 x v_bits bits.
+// this library's, described in include/sphkv.h):
+//   r[16] fp16 | vscale[16] fp16 | code planes (8 subtree blocks per token)
+//   | value rows (channels permuted for tensor-core fragments)
 #pragma once
 
 #include <cuda_fp16.h>
@@ -25,35 +24,27 @@ constexpr int kUpper = kD / 2 - 1;      // 63
 
 struct TierFmt {
     int b_leaf, b_up, v_bits;
-    int leaf_row, up_row, v_row;   // bytes per token row
-    int off_leaf, off_up, off_v;   // byte offsets inside the page
+    int code_row;     // code bytes per token (8 subtree blocks)
+    int v_row;        // value bytes per token
+    int off_codes, off_v;
     int page_bytes;
 };
 
-__host__ __device__ constexpr TierFmt make_fmt(int bl, int bu, int vb)
+__host__ __device__ constexpr TierFmt make_fmt(int bl, int bu, int vb, int code_row)
 {
-    return TierFmt{bl,
-                   bu,
-                   vb,
-                   kLeaves * bl / 8,
-                   (kUpper * bu + 127) / 128 * 16,
-                   kD * vb / 8,
-                   4 * kP,
-                   4 * kP + kP * (kLeaves * bl / 8),
-                   4 * kP + kP * (kLeaves * bl / 8) + kP * ((kUpper * bu + 127) / 128 * 16),
-                   4 * kP + kP * (kLeaves * bl / 8) + kP * ((kUpper * bu + 127) / 128 * 16) +
-                       kP * (kD * vb / 8)};
+    return TierFmt{bl, bu, vb, code_row, kD * vb / 8, 4 * kP, 4 * kP + kP * code_row,
+                   4 * kP + kP * code_row + kP * (kD * vb / 8)};
 }
 
 // Tier index 1..3 (0 = drop).
 template <int T>
 struct Tier;
 template <>
-struct Tier<1> { static constexpr TierFmt f = make_fmt(8, 8, 8); };
+struct Tier<1> { static constexpr TierFmt f = make_fmt(8, 8, 8, 128); };
 template <>
-struct Tier<2> { static constexpr TierFmt f = make_fmt(4, 6, 4); };
+struct Tier<2> { static constexpr TierFmt f = make_fmt(4, 6, 4, 80); };
 template <>
-struct Tier<3> { static constexpr TierFmt f = make_fmt(3, 4, 4); };
+struct Tier<3> { static constexpr TierFmt f = make_fmt(3, 4, 4, 56); };
 
 static_assert(Tier<1>::f.page_bytes == 4160, "T1 page");
 static_assert(Tier<2>::f.page_bytes == 2368, "T2 page");
@@ -61,6 +52,9 @@ static_assert(Tier<3>::f.page_bytes == 1984, "T3 page");
 static_assert(Tier<1>::f.page_bytes % 16 == 0 && Tier<2>::f.page_bytes % 16 == 0 &&
                   Tier<3>::f.page_bytes % 16 == 0,
               "pages must be 16-byte multiples for bulk copies");
+
+// Value row position p = 16g + 2m + h holds channel 16m + g + 8h.
+__host__ __device__ constexpr int v_channel_at(int p) { return 16 * ((p >> 1) & 7) + (p >> 4) + 8 * (p & 1); }
 
 __host__ __device__ inline int page_bytes_of(int t)
 {

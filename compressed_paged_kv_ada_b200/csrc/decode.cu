@@ -13,16 +13,26 @@
 //
 // Launch structure (three kernels on the caller's stream):
 //   plan   -- 1 CTA: unit_start[u] = pages before unit u = (b, g), u = b*H_kv+g.
-//   decode -- persistent, one 512-thread CTA per SM.  The flattened page range
+//   decode -- persistent, one 384-thread CTA per SM.  The flattened page range
 //             [0, P) is cut into n_cta equal pieces; a CTA walks the units its
-//             piece overlaps.  Its 16 warps take the unit's pages round robin;
+//             piece overlaps.  Its 12 warps take the unit's pages round robin;
 //             each warp bulk-copies a page (cp.async.bulk, mbarrier completion)
 //             into a 2-stage ring in shared memory while it computes the
-//             previous one.  A warp covers 4 tokens per pass, 8 lanes per
-//             token, each lane an 8-leaf subtree; the three top tree levels
-//             use shuffles that hand each lane a different query head.  The
-//             per-tier cos/sin tables sit in shared memory, replicated 16
-//             times so a half-warp's 64-bit lookups never share a bank.
+//             previous one.
+//             Logits: 4 tokens per pass, 8 lanes per token; lane s owns the
+//             8-leaf subtree s (one aligned code block) and all 4 query heads,
+//             so each cos/sin lookup serves 4 heads.  The three top tree levels
+//             use shuffles that leave each lane a different head.  Tables sit in
+//             shared memory as rows of 256 bytes per code: 16 lane replicas of
+//             (cos, sin) for the leaf grid and for the upper grid, so a half
+//             warp's 64-bit lookups never share a bank and the address is one
+//             byte permute.  (Packed f32x2 arithmetic would need {cos,cos} and
+//             {sin,sin} pairs, i.e. 16-byte lookups; measured on B200 that
+//             doubles shared-memory traffic and is slower.)
+//             Values: out^T[dims x heads] += V^T[dims x 16 tokens] P^T[16 x 4]
+//             on the tensor cores (mma.sync m16n8k16, f16 operands, fp32
+//             accumulators).  Value codes are exact in f16; the weights p*scale
+//             are split into f16 hi + lo parts (two MMAs), keeping ~22 bits.
 //   merge  -- one CTA per unit whose pages were split over several CTAs.
 #include "common.cuh"
 
@@ -30,23 +40,21 @@ namespace sphkv {
 namespace {
 
 constexpr int kG = 4;               // query heads per kv head
-constexpr int kWarps = 16;
+constexpr int kWarps = 12;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 2;
 constexpr int kStageBytes = Tier<1>::f.page_bytes;  // largest page
-constexpr int kRep = 16;            // LUT replicas (one per lane of a half warp)
 constexpr int kMinPagesPerCta = 64;
 constexpr int kPartStride = 132;    // floats per (slot, head): m, l, pad, pad, o[128]
 
-// LUT entries: leaf tables of T1/T2/T3 then upper tables of T1/T2/T3.
-constexpr int kLeafBase1 = 0, kLeafBase2 = 256, kLeafBase3 = 272;
-constexpr int kUpBase1 = 280, kUpBase2 = 536, kUpBase3 = 600;
-constexpr int kLutEntries = 616;
-
-constexpr int kLutBytes = kLutEntries * kRep * 8;
+// LUT: per tier, one 256-byte row per code: [leaf (cos,sin) x 16 replicas]
+// [upper (cos,sin) x 16 replicas].  Rows: T1 256, T2 64, T3 16.
+constexpr int kLutRow = 256;
+constexpr int kLutT1 = 0, kLutT2 = 256 * kLutRow, kLutT3 = kLutT2 + 64 * kLutRow;
+constexpr int kLutBytes = kLutT3 + 16 * kLutRow;
 constexpr int kStageOff = kLutBytes;
 constexpr int kPbufOff = kStageOff + kWarps * kStages * kStageBytes;
-constexpr int kPbufFloats = 16 * kG + kG;   // p*scale per (token, head), then alpha per head
+constexpr int kPbufFloats = 16 * kG + 2 * kG;   // p*scale per (token, head); alpha per head; pad
 constexpr int kBarOff = kPbufOff + kWarps * kPbufFloats * 4;
 constexpr int kSmemBytes = kBarOff + kWarps * kStages * 8;
 static_assert(kStageOff % 128 == 0 && kPbufOff % 16 == 0 && kBarOff % 8 == 0, "smem alignment");
@@ -57,17 +65,11 @@ static_assert((2 * kWarps * kG + kWarps * kG * kD) * 4 <= kWarps * kStages * kSt
 constexpr float kLn2 = 0.6931471805599453f;
 // log2(e) / sqrt(128): logits are kept in the log2 domain
 constexpr float kLogitScale = 0.12751743082459868f;
+// the value weights p * scale are multiplied by 2^12 before the f16 split
+constexpr float kPScale = 4096.0f;
+constexpr float kInvPScale = 1.0f / 4096.0f;
 
 constexpr long kWaitLimit = 1L << 22;
-
-template <int T>
-struct TierLut;
-template <>
-struct TierLut<1> { static constexpr int leaf = kLeafBase1, up = kUpBase1; };
-template <>
-struct TierLut<2> { static constexpr int leaf = kLeafBase2, up = kUpBase2; };
-template <>
-struct TierLut<3> { static constexpr int leaf = kLeafBase3, up = kUpBase3; };
 
 struct DecodeParams {
     const int32_t* page_offsets;
@@ -143,15 +145,6 @@ __device__ inline bool mbar_wait(uint32_t bar, uint32_t parity)
     return false;
 }
 
-__device__ inline uint32_t ld_u32(const uint8_t* p) { return *(const uint32_t*)p; }
-
-// 32 bits of a row's LSB-first bit stream starting at bit `pos` (row 4-byte aligned).
-__device__ inline uint32_t bits_at(const uint8_t* row, int pos)
-{
-    const uint32_t* w = (const uint32_t*)row + (pos >> 5);
-    return __funnelshift_r(w[0], w[1], pos & 31);
-}
-
 // ---------------------------------------------------------------- plan --
 __global__ void __launch_bounds__(1024) plan_kernel(DecodeParams p)
 {
@@ -225,84 +218,123 @@ __device__ inline int32_t cta_bound(int c, int32_t P, int n_cta)
 
 // ------------------------------------------------------------- page work --
 struct WarpState {
-    float m;        // running max (log2 domain) of this lane's head
-    float l;        // running sum of this lane's tokens
-    float o[kG][4]; // out accumulators: 4 heads x dims 4*lane .. 4*lane+3
+    float m;             // running max (log2 domain) of this lane's head
+    float l;             // running sum of this lane's tokens
+    float acc[8][4];     // MMA accumulators: tile m = dims 16m..16m+15
 };
 
-__device__ inline float2 lut_get(const float2* lut, int entry, int lane)
+// LUT byte offsets (tier base | code << 8 | replica << 3) of the 8 leaf and 8
+// upper codes of one subtree block.  base_rep = tier base | (lane & 15) << 3.
+template <int T>
+__device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uint32_t base_rep, uint32_t (&lo)[8],
+                                              uint32_t (&uo)[8])
 {
-    return lut[entry * kRep + (lane & (kRep - 1))];
+    if (T == 1) {   // byte codes: one permute places the code in bits 8..15
+        const uint4 w = *(const uint4*)(codes + blk * 16);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            lo[j] = __byte_perm(w.x, base_rep, 0x7604 | (j << 4));
+            lo[4 + j] = __byte_perm(w.y, base_rep, 0x7604 | (j << 4));
+            uo[j] = __byte_perm(w.z, base_rep, 0x7604 | (j << 4));
+            uo[4 + j] = __byte_perm(w.w, base_rep, 0x7604 | (j << 4));
+        }
+    } else if (T == 2) {
+        const uint2 w = *(const uint2*)(codes + blk * 8);
+        const uint32_t h = *(const uint16_t*)(codes + kP * 64 + blk * 2);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            lo[j] = (((w.x >> (4 * j)) & 15u) << 8) | base_rep;
+            uo[j] = (((w.y >> (4 * j)) & 15u) << 8) | (((h >> (2 * j)) & 3u) << 12) | base_rep;
+        }
+    } else {
+        const uint32_t u = *(const uint32_t*)(codes + blk * 4);
+        const uint32_t l2 = *(const uint16_t*)(codes + kP * 32 + blk * 2);
+        const uint32_t l1 = codes[kP * 48 + blk];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            lo[j] = (((l2 >> (2 * j)) & 3u) << 8) | (((l1 >> j) & 1u) << 10) | base_rep;
+            uo[j] = (((u >> (4 * j)) & 15u) << 8) | base_rep;
+        }
+    }
 }
 
-// One page of tier T already staged in shared memory at `pg`.
-template <int T>
-__device__ __forceinline__ void process_page(const uint8_t* pg, int valid, const float (&qr)[kG][16],
-                                             const float2* lut, float* pbuf, int lane,
-                                             WarpState& st)
+// (cos, sin) of a leaf or an upper code at LUT byte offset `off`.
+__device__ __forceinline__ float2 lut_leaf(const uint8_t* smem, uint32_t off)
 {
-    constexpr TierFmt F = Tier<T>::f;
-    constexpr int LB = TierLut<T>::leaf, UB = TierLut<T>::up;
-    constexpr uint32_t LM = (1u << F.b_leaf) - 1, UM = (1u << F.b_up) - 1;
+    return *(const float2*)(smem + off);
+}
+__device__ __forceinline__ float2 lut_up(const uint8_t* smem, uint32_t off)
+{
+    return *(const float2*)(smem + 128 + off);
+}
+
+// Two halves packed as f16x2: `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi)
+{
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *(const uint32_t*)&h;
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// One page of tier `tier` already staged in shared memory at `pg`.  Only the
+// code extraction and the value conversion depend on the tier; the tree, the
+// softmax and the MMAs are one copy of code for all tiers (a small kernel keeps
+// the instruction cache warm while warps interleave pages of different tiers).
+__device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int valid, const float (&qr)[kG][16],
+                                             const uint8_t* smem, float* pbuf, int lane, WarpState& st)
+{
     const unsigned full = 0xffffffffu;
     const int k = lane >> 3, s = lane & 7;
     const int head = (s & 1) * 2 + ((s >> 1) & 1);   // head held after the shuffle levels
-    float lg[4];
-#pragma unroll
+    const uint32_t base_rep = (uint32_t)(tier == 1 ? kLutT1 : tier == 2 ? kLutT2 : kLutT3) | ((uint32_t)(lane & 15) << 3);
+    const uint8_t* codes = pg + Tier<1>::f.off_codes;
+    float lg0 = -INFINITY, lg1 = -INFINITY, lg2 = -INFINITY, lg3 = -INFINITY;
+#pragma unroll 1
     for (int pass = 0; pass < 4; ++pass) {
         const int t = pass * 4 + k;
-        const uint8_t* lrow = pg + F.off_leaf + t * F.leaf_row;
-        const uint8_t* urow = pg + F.off_up + t * F.up_row;
-        // leaf codes of leaves 8s .. 8s+7
-        uint32_t lc0, lc1 = 0;
-        if (F.b_leaf == 8) {
-            lc0 = ld_u32(lrow + 8 * s);
-            lc1 = ld_u32(lrow + 8 * s + 4);
-        } else if (F.b_leaf == 4) {
-            lc0 = ld_u32(lrow + 4 * s);
-        } else {
-            lc0 = bits_at(lrow, 8 * s * F.b_leaf);
-        }
-        const uint32_t u1 = bits_at(urow, (4 * s) * F.b_up);          // level 1: nodes 4s..4s+3
-        const uint32_t u2 = bits_at(urow, (32 + 2 * s) * F.b_up);     // level 2: nodes 2s, 2s+1
-        const uint32_t u3 = bits_at(urow, (48 + s) * F.b_up);         // level 3: node s
-        const uint32_t u4 = bits_at(urow, (56 + (s >> 1)) * F.b_up);  // level 4
-        const uint32_t u5 = bits_at(urow, (60 + (s >> 2)) * F.b_up);  // level 5
-        const uint32_t u6 = bits_at(urow, 62 * F.b_up);               // root
+        uint32_t lo[8], uo[8];
+        if (tier == 1) block_offsets<1>(codes, t * 8 + s, base_rep, lo, uo);
+        else if (tier == 2) block_offsets<2>(codes, t * 8 + s, base_rep, lo, uo);
+        else block_offsets<3>(codes, t * 8 + s, base_rep, lo, uo);
+        // top codes: block i carries top node i (level 4 nodes 0..3, level 5
+        // nodes 0..1, root); lane s needs nodes s>>1, 4 + (s>>2) and 6
+        const uint32_t o4 = __shfl_sync(full, uo[7], (lane & ~7) | (s >> 1));
+        const uint32_t o5 = __shfl_sync(full, uo[7], (lane & ~7) | (4 + (s >> 2)));
+        const uint32_t o6 = __shfl_sync(full, uo[7], (lane & ~7) | 6);
+        // subtree of 8 leaves, 4 heads
         float S1[4][kG];
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-            uint32_t ca, cb;
-            if (F.b_leaf == 8) {
-                const uint32_t src = m < 2 ? lc0 : lc1;
-                ca = (src >> (16 * (m & 1))) & LM;
-                cb = (src >> (16 * (m & 1) + 8)) & LM;
-            } else {
-                ca = (lc0 >> ((2 * m) * F.b_leaf)) & LM;
-                cb = (lc0 >> ((2 * m + 1) * F.b_leaf)) & LM;
-            }
-            const float2 fa = lut_get(lut, LB + ca, lane);
-            const float2 fb = lut_get(lut, LB + cb, lane);
-            const float2 fu = lut_get(lut, UB + ((u1 >> (m * F.b_up)) & UM), lane);
+            const float2 fa = lut_leaf(smem, lo[2 * m]);
+            const float2 fb = lut_leaf(smem, lo[2 * m + 1]);
+            const float2 fu = lut_up(smem, uo[m]);
 #pragma unroll
             for (int h = 0; h < kG; ++h) {
-                const float L = qr[h][4 * m] * fa.x + qr[h][4 * m + 1] * fa.y;
-                const float R = qr[h][4 * m + 2] * fb.x + qr[h][4 * m + 3] * fb.y;
-                S1[m][h] = fu.x * L + fu.y * R;
+                const float L = fmaf(qr[h][4 * m + 1], fa.y, qr[h][4 * m] * fa.x);
+                const float R = fmaf(qr[h][4 * m + 3], fb.y, qr[h][4 * m + 2] * fb.x);
+                S1[m][h] = fmaf(fu.y, R, fu.x * L);
             }
         }
         float S2[2][kG];
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-            const float2 fu = lut_get(lut, UB + ((u2 >> (m * F.b_up)) & UM), lane);
+        for (int n = 0; n < 2; ++n) {
+            const float2 fu = lut_up(smem, uo[4 + n]);
 #pragma unroll
-            for (int h = 0; h < kG; ++h) S2[m][h] = fu.x * S1[2 * m][h] + fu.y * S1[2 * m + 1][h];
+            for (int h = 0; h < kG; ++h) S2[n][h] = fmaf(fu.y, S1[2 * n + 1][h], fu.x * S1[2 * n][h]);
         }
         float S3[kG];
         {
-            const float2 fu = lut_get(lut, UB + (u3 & UM), lane);
+            const float2 fu = lut_up(smem, uo[6]);
 #pragma unroll
-            for (int h = 0; h < kG; ++h) S3[h] = fu.x * S2[0][h] + fu.y * S2[1][h];
+            for (int h = 0; h < kG; ++h) S3[h] = fmaf(fu.y, S2[1][h], fu.x * S2[0][h]);
         }
         // level 4: lanes s, s^1 hold sibling subtrees; even lane keeps heads 0,1
         const bool odd = s & 1;
@@ -310,29 +342,34 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int valid, const
         const float r1 = __shfl_xor_sync(full, odd ? S3[1] : S3[3], 1);
         float T0, T1;
         {
-            const float2 fu = lut_get(lut, UB + (u4 & UM), lane);
-            T0 = fu.x * (odd ? r0 : S3[0]) + fu.y * (odd ? S3[2] : r0);
-            T1 = fu.x * (odd ? r1 : S3[1]) + fu.y * (odd ? S3[3] : r1);
+            const float2 fu = lut_up(smem, o4);
+            T0 = fmaf(fu.y, odd ? S3[2] : r0, fu.x * (odd ? r0 : S3[0]));
+            T1 = fmaf(fu.y, odd ? S3[3] : r1, fu.x * (odd ? r1 : S3[1]));
         }
         // level 5: lanes s, s^2; bit1 = 0 keeps the first of the pair
         const bool hi1 = (s >> 1) & 1;
         const float r2 = __shfl_xor_sync(full, hi1 ? T0 : T1, 2);
         float U;
         {
-            const float2 fu = lut_get(lut, UB + (u5 & UM), lane);
-            U = fu.x * (hi1 ? r2 : T0) + fu.y * (hi1 ? T1 : r2);
+            const float2 fu = lut_up(smem, o5);
+            U = fmaf(fu.y, hi1 ? T1 : r2, fu.x * (hi1 ? r2 : T0));
         }
         // root: lanes s, s^4 (both end with the same value)
         const bool right = (s >> 2) & 1;
         const float r3 = __shfl_xor_sync(full, U, 4);
         float S;
         {
-            const float2 fu = lut_get(lut, UB + (u6 & UM), lane);
-            S = fu.x * (right ? r3 : U) + fu.y * (right ? U : r3);
+            const float2 fu = lut_up(smem, o6);
+            S = fmaf(fu.y, right ? U : r3, fu.x * (right ? r3 : U));
         }
         const float rr = __half2float(((const __half*)pg)[t]);
-        lg[pass] = t < valid ? rr * S * kLogitScale : -INFINITY;
+        const float lv = t < valid ? rr * S * kLogitScale : -INFINITY;
+        lg0 = pass == 0 ? lv : lg0;
+        lg1 = pass == 1 ? lv : lg1;
+        lg2 = pass == 2 ? lv : lg2;
+        lg3 = pass == 3 ? lv : lg3;
     }
+    const float lg[4] = {lg0, lg1, lg2, lg3};
     // online softmax for this lane's head (lanes k = 0..3 share it)
     float pm = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
     pm = fmaxf(pm, __shfl_xor_sync(full, pm, 8));
@@ -346,35 +383,106 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int valid, const
     for (int pass = 0; pass < 4; ++pass) {
         const float pv = exp2f(lg[pass] - m_new);
         psum += pv;
-        if (s < 4) pbuf[(pass * 4 + k) * kG + head] = pv * __half2float(vs[pass * 4 + k]);
+        const int t = pass * 4 + k;   // slots past `valid` may hold stale scales: weight exactly 0
+        if (s < 4) pbuf[t * kG + head] = t < valid ? pv * __half2float(vs[t]) * kPScale : 0.f;
     }
     st.l = st.l * alpha + psum;
     if (lane < 4) pbuf[16 * kG + head] = alpha;
     __syncwarp();
-    const float4 al = *(const float4*)(pbuf + 16 * kG);
-    const float a4[kG] = {al.x, al.y, al.z, al.w};
+
+    // values on the tensor cores.  Thread (g, c): B columns = head g (g < 4),
+    // rows = tokens 2c, 2c+1 (b0) and 2c+8, 2c+9 (b1); accumulator columns =
+    // heads 2c, 2c+1.
+    const int g = lane >> 2, c = lane & 3;
+    {
+        const float2 al = *(const float2*)(pbuf + 16 * kG + 2 * (c & 1));
 #pragma unroll
-    for (int h = 0; h < kG; ++h)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) st.o[h][i] *= a4[h];
-    const uint8_t* vrow0 = pg + F.off_v;
-    for (int t = 0; t < valid; ++t) {
-        const float4 w = *(const float4*)(pbuf + t * kG);
-        float v[4];
-        if (F.v_bits == 8) {
-            const uint32_t x = ld_u32(vrow0 + t * F.v_row + 4 * lane);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) v[i] = (float)((int32_t)(x << (24 - 8 * i)) >> 24);
-        } else {
-            const uint32_t x = *(const uint16_t*)(vrow0 + t * F.v_row + 2 * lane);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) v[i] = (float)((int32_t)(x << (28 - 4 * i)) >> 28);
+        for (int m = 0; m < 8; ++m) {
+            st.acc[m][0] *= al.x;
+            st.acc[m][1] *= al.y;
+            st.acc[m][2] *= al.x;
+            st.acc[m][3] *= al.y;
         }
-        const float wv[kG] = {w.x, w.y, w.z, w.w};
+    }
+    uint32_t bh0 = 0, bh1 = 0, bl0 = 0, bl1 = 0;
+    if (g < kG) {
+        const float p0 = pbuf[(2 * c) * kG + g], p1 = pbuf[(2 * c + 1) * kG + g];
+        const float p2 = pbuf[(2 * c + 8) * kG + g], p3 = pbuf[(2 * c + 9) * kG + g];
+        const __half2 h01 = __floats2half2_rn(p0, p1), h23 = __floats2half2_rn(p2, p3);
+        bh0 = *(const uint32_t*)&h01;
+        bh1 = *(const uint32_t*)&h23;
+        bl0 = pack_h2(p0 - __low2float(h01), p1 - __high2float(h01));
+        bl1 = pack_h2(p2 - __low2float(h23), p3 - __high2float(h23));
+    }
+    // rows of tokens 2c, 2c+1, 2c+8, 2c+9 at positions 16g..16g+15; tokens past
+    // `valid` carry weight 0 (their rows may hold anything finite)
+    if (tier == 1) {
+        constexpr TierFmt F = Tier<1>::f;
+        const uint8_t* vrow = pg + F.off_v;
+        const __half2 bias = __floats2half2_rn(-1152.f, -1152.f);
+        // chunk g of row r sits at chunk g ^ (r & 6); r & 6 = 2c for all four rows
+        const int ch = 16 * (g ^ (2 * c));
+        const uint4 X = *(const uint4*)(vrow + (2 * c) * F.v_row + ch);
+        const uint4 Y = *(const uint4*)(vrow + (2 * c + 1) * F.v_row + ch);
+        const uint4 Z = *(const uint4*)(vrow + (2 * c + 8) * F.v_row + ch);
+        const uint4 W = *(const uint4*)(vrow + (2 * c + 9) * F.v_row + ch);
+        const uint32_t xs[4] = {X.x ^ 0x80808080u, X.y ^ 0x80808080u, X.z ^ 0x80808080u, X.w ^ 0x80808080u};
+        const uint32_t ys[4] = {Y.x ^ 0x80808080u, Y.y ^ 0x80808080u, Y.z ^ 0x80808080u, Y.w ^ 0x80808080u};
+        const uint32_t zs[4] = {Z.x ^ 0x80808080u, Z.y ^ 0x80808080u, Z.z ^ 0x80808080u, Z.w ^ 0x80808080u};
+        const uint32_t ws[4] = {W.x ^ 0x80808080u, W.y ^ 0x80808080u, W.z ^ 0x80808080u, W.w ^ 0x80808080u};
 #pragma unroll
-        for (int h = 0; h < kG; ++h)
+        for (int m = 0; m < 8; ++m) {
+            const int wi = m >> 1, b = 2 * (m & 1);   // byte b (h = 0) and b + 1 (h = 1) of word wi
+            // result byte 0 <- low token's byte, byte 2 <- high token's byte;
+            // | 0x6400 makes f16 1024 + u, u = code + 128
+            const uint32_t sel0 = (uint32_t)(b | ((4 + b) << 8));
+            const uint32_t sel1 = (uint32_t)((b + 1) | ((5 + b) << 8));
+            uint32_t a[4];
+            a[0] = (__byte_perm(xs[wi], ys[wi], sel0) & 0x00FF00FFu) | 0x64006400u;
+            a[1] = (__byte_perm(xs[wi], ys[wi], sel1) & 0x00FF00FFu) | 0x64006400u;
+            a[2] = (__byte_perm(zs[wi], ws[wi], sel0) & 0x00FF00FFu) | 0x64006400u;
+            a[3] = (__byte_perm(zs[wi], ws[wi], sel1) & 0x00FF00FFu) | 0x64006400u;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) st.o[h][i] = fmaf(wv[h], v[i], st.o[h][i]);
+            for (int i = 0; i < 4; ++i) {
+                __half2 hv = __hadd2(*(const __half2*)&a[i], bias);
+                a[i] = *(const uint32_t*)&hv;
+            }
+            mma_16816(st.acc[m], a, bh0, bh1);
+            mma_16816(st.acc[m], a, bl0, bl1);
+        }
+    } else {   // T2 and T3 share the int4 row format
+        const uint8_t* vrow = pg + (tier == 2 ? Tier<2>::f.off_v : Tier<3>::f.off_v);
+        const __half2 bias = __floats2half2_rn(-1032.f, -1032.f);
+        // tokens 2i, 2i+1 share a 128-byte block; chunk g ^ (2i & 6) holds 8
+        // bytes of each.  Pairs c and c + 4 both give 2i & 6 = 2c.
+        const int ch = 16 * (g ^ (2 * c));
+        const uint4 XY = *(const uint4*)(vrow + c * 128 + ch);
+        const uint4 ZW = *(const uint4*)(vrow + (c + 4) * 128 + ch);
+        const uint2 X = make_uint2(XY.x, XY.y), Y = make_uint2(XY.z, XY.w);
+        const uint2 Z = make_uint2(ZW.x, ZW.y), W = make_uint2(ZW.z, ZW.w);
+        const uint32_t xs[2] = {X.x ^ 0x88888888u, X.y ^ 0x88888888u};
+        const uint32_t ys[2] = {Y.x ^ 0x88888888u, Y.y ^ 0x88888888u};
+        const uint32_t zs[2] = {Z.x ^ 0x88888888u, Z.y ^ 0x88888888u};
+        const uint32_t ws[2] = {W.x ^ 0x88888888u, W.y ^ 0x88888888u};
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int wi = m >> 2, b = m & 3;   // byte m: low nibble h = 0, high nibble h = 1
+            const uint32_t sel = (uint32_t)(b | ((4 + b) << 8));
+            const uint32_t xy = __byte_perm(xs[wi], ys[wi], sel);
+            const uint32_t zw = __byte_perm(zs[wi], ws[wi], sel);
+            uint32_t a[4];
+            a[0] = (xy & 0x000F000Fu) | 0x64006400u;
+            a[1] = ((xy >> 4) & 0x000F000Fu) | 0x64006400u;
+            a[2] = (zw & 0x000F000Fu) | 0x64006400u;
+            a[3] = ((zw >> 4) & 0x000F000Fu) | 0x64006400u;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                __half2 hv = __hadd2(*(const __half2*)&a[i], bias);
+                a[i] = *(const uint32_t*)&hv;
+            }
+            mma_16816(st.acc[m], a, bh0, bh1);
+            mma_16816(st.acc[m], a, bl0, bl1);
+        }
     }
     __syncwarp();
 }
@@ -383,24 +491,30 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int valid, const
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
 {
     extern __shared__ __align__(128) uint8_t smem[];
-    float2* lut = (float2*)smem;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const unsigned full = 0xffffffffu;
 
-    // cos/sin tables: leaf grids c*2pi/2^b, upper grids c*(pi/2)/(2^b-1)
-    for (int e = tid; e < kLutEntries; e += kThreads) {
-        double a;   // angle / pi
-        if (e < kLeafBase2) a = (double)e / 128.0;
-        else if (e < kLeafBase3) a = (double)(e - kLeafBase2) / 8.0;
-        else if (e < kUpBase1) a = (double)(e - kLeafBase3) / 4.0;
-        else if (e < kUpBase2) a = (double)(e - kUpBase1) / 510.0;
-        else if (e < kUpBase3) a = (double)(e - kUpBase2) / 126.0;
-        else a = (double)(e - kUpBase3) / 30.0;
-        double sn, cs;
-        sincospi(a, &sn, &cs);
-        const float2 v = make_float2((float)cs, (float)sn);
+    // cos/sin tables, one 256-byte row per code: leaf grid c*2pi/2^b_leaf in
+    // bytes 0..127, upper grid c*(pi/2)/(2^b_up-1) in bytes 128..255, each
+    // entry replicated for the 16 lanes of a half warp
+    {
+        constexpr int kRows = 256 + 64 + 16;
+        for (int e = tid; e < 2 * kRows; e += kThreads) {
+            const int row = e >> 1, upper = e & 1;
+            int tier_base, code, nleaf, nup;
+            if (row < 256) { tier_base = kLutT1; code = row; nleaf = 256; nup = 256; }
+            else if (row < 320) { tier_base = kLutT2; code = row - 256; nleaf = 16; nup = 64; }
+            else { tier_base = kLutT3; code = row - 320; nleaf = 8; nup = 16; }
+            double a = 0.0;   // angle / pi
+            if (!upper && code < nleaf) a = 2.0 * code / nleaf;
+            if (upper && code < nup) a = 0.5 * code / (nup - 1);
+            double sn, cs;
+            sincospi(a, &sn, &cs);
+            const float2 v = make_float2((float)cs, (float)sn);
+            float2* dst = (float2*)(smem + tier_base + code * kLutRow + upper * 128);
 #pragma unroll
-        for (int r = 0; r < kRep; ++r) lut[e * kRep + r] = v;
+            for (int r = 0; r < 16; ++r) dst[r] = v;
+        }
     }
     uint8_t* stage = smem + kStageOff + w * kStages * kStageBytes;
     float* pbuf = (float*)(smem + kPbufOff) + w * kPbufFloats;
@@ -431,7 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
         const int len = p.seq_lens[b];
         const int32_t* ptab = p.page_table + (int64_t)g * p.total_pages + first;
 
-        // this lane's query slice: dims 16s .. 16s+15 of heads 4g .. 4g+3
+        // this lane's query slice: dims 16s .. 16s+15 of heads 4g .. 4g+3, as
+        // pairs of heads {4g + 2hp, 4g + 2hp + 1}
         float qr[kG][16];
         {
             const int s = lane & 7;
@@ -452,54 +567,59 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
         st.m = -INFINITY;
         st.l = 0.f;
 #pragma unroll
-        for (int h = 0; h < kG; ++h)
+        for (int m = 0; m < 8; ++m)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) st.o[h][i] = 0.f;
+            for (int i = 0; i < 4; ++i) st.acc[m][i] = 0.f;
 
-        // this warp's pages: pa + w + 16 i.  Entries are read 32 at a time.
-        int ebase = 0;
-        int32_t ent = 0;
-        uint32_t mask = 0;
-        auto refill = [&]() {
-            const int32_t lp = pa + w + kWarps * (ebase + lane);
-            ent = lp < pe ? ptab[lp] : 0;
-            int t = entry_tier(ent);
+        // this warp's pages: pa + w + kWarps*i.  Entries are read 32 at a time.
+        struct Cursor {
+            int ebase;
+            int32_t ent;
+            uint32_t mask;
+        };
+        auto refill = [&](Cursor& cu) {
+            const int32_t lp = pa + w + kWarps * (cu.ebase + lane);
+            cu.ent = lp < pe ? ptab[lp] : 0;
+            const int t = entry_tier(cu.ent);
             bool ok = t != 0;
-            if (ok && entry_page(ent) >= p.pool_pages[t]) {
+            if (ok && entry_page(cu.ent) >= p.pool_pages[t]) {
                 report(p.status, SPHKV_ERR_DATA);
                 ok = false;
             }
-            mask = __ballot_sync(full, ok);
+            cu.mask = __ballot_sync(full, ok);
         };
-        auto next = [&](int32_t& lp, int32_t& e) -> bool {
-            while (mask == 0) {
-                ebase += 32;
-                if (pa + w + kWarps * ebase >= pe) return false;
-                refill();
+        auto advance = [&](Cursor& cu, int32_t& lp, int32_t& e) -> bool {
+            while (cu.mask == 0) {
+                cu.ebase += 32;
+                if (pa + w + kWarps * cu.ebase >= pe) return false;
+                refill(cu);
             }
-            const int j = __ffs(mask) - 1;
-            mask &= mask - 1;
-            lp = pa + w + kWarps * (ebase + j);
-            e = __shfl_sync(full, ent, j);
+            const int j = __ffs(cu.mask) - 1;
+            cu.mask &= cu.mask - 1;
+            lp = pa + w + kWarps * (cu.ebase + j);
+            e = __shfl_sync(full, cu.ent, j);
             return true;
+        };
+        auto page_src = [&](int32_t e) -> const uint8_t* {
+            const int t = entry_tier(e);
+            return p.pool[t] + entry_page(e) * (int64_t)page_bytes_of(t);
         };
         auto issue = [&](int stg, int32_t e) {
             if (lane == 0) {
-                const int t = entry_tier(e);
-                const uint32_t bytes = (uint32_t)page_bytes_of(t);
-                const uint8_t* src = p.pool[t] + entry_page(e) * (int64_t)bytes;
+                const uint32_t bytes = (uint32_t)page_bytes_of(entry_tier(e));
                 fence_proxy_async();
                 mbar_expect_tx(bar0 + 8 * stg, bytes);
-                bulk_g2s(smem_u32(stage + stg * kStageBytes), src, bytes, bar0 + 8 * stg);
+                bulk_g2s(smem_u32(stage + stg * kStageBytes), page_src(e), bytes, bar0 + 8 * stg);
             }
         };
-        refill();
+        Cursor cur_c{0, 0, 0u};
+        refill(cur_c);
         int32_t lp_cur = 0, e_cur = 0, lp_nxt = 0, e_nxt = 0;
-        bool have_cur = next(lp_cur, e_cur);
+        bool have_cur = advance(cur_c, lp_cur, e_cur);
         int cur = 0;
         if (have_cur) issue(0, e_cur);
         while (have_cur) {
-            const bool have_nxt = next(lp_nxt, e_nxt);
+            const bool have_nxt = advance(cur_c, lp_nxt, e_nxt);
             if (have_nxt) issue(cur ^ 1, e_nxt);
             const bool ok = mbar_wait(bar0 + 8 * cur, (phase >> cur) & 1);
             phase ^= 1u << cur;
@@ -515,9 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
             const uint8_t* pg = stage + cur * kStageBytes;
             const int valid = min(kP, len - lp_cur * kP);
             const int t = entry_tier(e_cur);
-            if (t == 1) process_page<1>(pg, valid, qr, lut, pbuf, lane, st);
-            else if (t == 2) process_page<2>(pg, valid, qr, lut, pbuf, lane, st);
-            else process_page<3>(pg, valid, qr, lut, pbuf, lane, st);
+            process_page(pg, t, valid, qr, smem, pbuf, lane, st);
             cur ^= 1;
             lp_cur = lp_nxt;
             e_cur = e_nxt;
@@ -536,14 +654,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
                 ms_m[w * kG + head] = st.m;
                 ms_l[w * kG + head] = lt;
             }
+            // accumulator (tile m, i): dim 16m + g + 8*(i >> 1), head 2c + (i & 1)
+            const int gq = lane >> 2, cq = lane & 3;
+            if (cq < 2) {
 #pragma unroll
-            for (int h = 0; h < kG; ++h)
-                *(float4*)(ms_o + (w * kG + h) * kD + 4 * lane) =
-                    make_float4(st.o[h][0], st.o[h][1], st.o[h][2], st.o[h][3]);
+                for (int m = 0; m < 8; ++m)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        ms_o[(w * kG + 2 * cq + (i & 1)) * kD + 16 * m + gq + 8 * (i >> 1)] = st.acc[m][i];
+            }
         }
         __syncthreads();
-        {
-            const int h = tid >> 7, dim = tid & (kD - 1);
+        for (int idx = tid; idx < kG * kD; idx += kThreads) {
+            const int h = idx >> 7, dim = idx & (kD - 1);
             float M = -INFINITY;
 #pragma unroll
             for (int ww = 0; ww < kWarps; ++ww) M = fmaxf(M, ms_m[ww * kG + h]);
@@ -560,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
             }
             if (pa == 0 && seg_end == ue) {   // the whole unit: final result
                 const int64_t row = (int64_t)b * p.H_q + g * kG + h;
-                p.out[row * kD + dim] = L > 0.f ? O / L : 0.f;
+                p.out[row * kD + dim] = L > 0.f ? O * kInvPScale / L : 0.f;
                 if (dim == 0) p.lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
             } else {
                 float* part = p.partial + ((int64_t)(blockIdx.x + u) * kG + h) * kPartStride;
@@ -614,7 +737,7 @@ __global__ void __launch_bounds__(kG * kD) merge_kernel(DecodeParams p)
             O += part[4 + dim] * sc;
         }
     }
-    p.out[row * kD + dim] = L > 0.f ? O / L : 0.f;
+    p.out[row * kD + dim] = L > 0.f ? O * kInvPScale / L : 0.f;
     if (dim == 0) p.lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
 }
 

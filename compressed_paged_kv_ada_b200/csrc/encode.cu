@@ -69,19 +69,12 @@ __device__ inline int upper_code(double ss_l, double ss_r, int b)
     return (int)t;
 }
 
-// 32-bit word w of a bit stream of n codes of b bits each, LSB first.
-__device__ inline uint32_t stream_word(const uint8_t* codes, int n, int b, int w)
+// Upper code j of subtree block s (see include/sphkv.h): level-1 nodes
+// 4s..4s+3, level-2 nodes 2s, 2s+1, level-3 node s, then top node s.
+__device__ inline uint32_t block_up(const uint8_t* up, int s, int j)
 {
-    uint32_t word = 0;
-    int first = (32 * w) / b;
-    int last = (32 * w + 31) / b;
-    if (last > n - 1) last = n - 1;
-    for (int i = first; i <= last; ++i) {
-        int sh = i * b - 32 * w;
-        uint64_t c = codes[i];
-        word |= sh >= 0 ? (uint32_t)(c << sh) : (uint32_t)(c >> (-sh));
-    }
-    return word;
+    return j < 4 ? up[4 * s + j] : j < 6 ? up[32 + 2 * s + (j - 4)] : j == 6 ? up[48 + s]
+                                                                            : (s < 7 ? up[56 + s] : 0u);
 }
 
 template <int T>
@@ -129,23 +122,75 @@ __device__ void encode_token(const EncParams& p, int64_t i, int g, uint8_t* page
         double t = s == 0.0 ? 0.0 : rint(__ddiv_rn(v[c], s));
         q[c] = (int)fmin(fmax(t, -Q), Q);
     }
+    __shared__ int8_t s_vq[kEncWarps][kD];
+    int8_t* vq = s_vq[threadIdx.x >> 5];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) vq[4 * lane + c] = (int8_t)q[c];
     __syncwarp();
-    // rows
-    uint8_t* lrow = page + F.off_leaf + slot * F.leaf_row;
-    uint8_t* urow = page + F.off_up + slot * F.up_row;
-    uint8_t* vrow = page + F.off_v + slot * F.v_row;
-    if (lane < F.leaf_row / 4)
-        ((uint32_t*)lrow)[lane] = stream_word(sleaf, kLeaves, F.b_leaf, lane);
-    if (lane < F.up_row / 4)
-        ((uint32_t*)urow)[lane] = stream_word(sup, kUpper, F.b_up, lane);
-    if (F.v_bits == 8) {
-        uint32_t w = (uint32_t)(q[0] & 0xff) | ((uint32_t)(q[1] & 0xff) << 8) |
-                     ((uint32_t)(q[2] & 0xff) << 16) | ((uint32_t)(q[3] & 0xff) << 24);
-        ((uint32_t*)vrow)[lane] = w;
-    } else {
-        uint16_t w = (uint16_t)((q[0] & 0xf) | ((q[1] & 0xf) << 4) | ((q[2] & 0xf) << 8) |
-                                ((q[3] & 0xf) << 12));
-        ((uint16_t*)vrow)[lane] = w;
+    // code blocks: 8 per token; lane l writes 32-bit word l of the token's blocks
+    uint8_t* codes = page + F.off_codes;
+    if (T == 1) {   // block s = 16 bytes: 8 leaf codes then 8 upper codes
+        const int s = lane >> 2, w = lane & 3;
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int j = 4 * (w & 1) + b;
+            const uint32_t code = w < 2 ? sleaf[8 * s + j] : block_up(sup, s, j);
+            word |= code << (8 * b);
+        }
+        ((uint32_t*)codes)[slot * 32 + lane] = word;
+    } else if (T == 2) {   // u32 leaf nibbles, u32 upper low nibbles | u16 upper high bits
+        if (lane < 16) {
+            const int s = lane >> 1, w = lane & 1;
+            uint32_t word = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                word |= (w == 0 ? (uint32_t)sleaf[8 * s + j] : (block_up(sup, s, j) & 15u)) << (4 * j);
+            ((uint32_t*)codes)[slot * 16 + lane] = word;
+        } else if (lane < 24) {
+            const int s = lane - 16;
+            uint32_t h = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h |= (block_up(sup, s, j) >> 4) << (2 * j);
+            ((uint16_t*)(codes + kP * 64))[slot * 8 + s] = (uint16_t)h;
+        }
+    } else {   // u32 upper nibbles | u16 leaf low 2 bits | u8 leaf high bit
+        if (lane < 8) {
+            const int s = lane;
+            uint32_t word = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) word |= block_up(sup, s, j) << (4 * j);
+            ((uint32_t*)codes)[slot * 8 + s] = word;
+        } else if (lane < 16) {
+            const int s = lane - 8;
+            uint32_t lo = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) lo |= ((uint32_t)sleaf[8 * s + j] & 3u) << (2 * j);
+            ((uint16_t*)(codes + kP * 32))[slot * 8 + s] = (uint16_t)lo;
+        } else if (lane < 24) {
+            const int s = lane - 16;
+            uint32_t hi = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) hi |= ((uint32_t)sleaf[8 * s + j] >> 2) << j;
+            (codes + kP * 48)[slot * 8 + s] = (uint8_t)hi;
+        }
+    }
+    // value row: position p holds channel v_channel_at(p); 16-byte chunks are
+    // swizzled (see include/sphkv.h) so the decoder's fragment loads are
+    // bank-conflict free
+    uint8_t* vsec = page + F.off_v;
+    if (F.v_bits == 8) {   // lane l: positions 4l..4l+3 = chunk l>>2, bytes 4(l&3)..
+        uint32_t w = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) w |= ((uint32_t)(uint8_t)vq[v_channel_at(4 * lane + b)]) << (8 * b);
+        const int g = lane >> 2;
+        *(uint32_t*)(vsec + slot * 128 + 16 * (g ^ (slot & 6)) + 4 * (lane & 3)) = w;
+    } else if (lane < 16) {   // lane l: positions 8l..8l+7 = chunk l>>1, bytes 4(l&1)..
+        uint32_t w = 0;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) w |= ((uint32_t)vq[v_channel_at(8 * lane + b)] & 15u) << (4 * b);
+        const int g = lane >> 1, i = slot >> 1;
+        *(uint32_t*)(vsec + i * 128 + 16 * (g ^ ((2 * i) & 6)) + 8 * (slot & 1) + 4 * (lane & 1)) = w;
     }
     if (lane == 0) {
         __half r16 = __double2half(sqrt(ss));

@@ -41,13 +41,29 @@
  *
  *  Tiers: T1 (b_leaf 8, b_up 8, int8 V, 4160 B/page), T2 (4, 6, int4, 2368 B),
  *  T3 (3, 4, int4, 1984 B), or drop (no storage, excluded from the softmax).
- *  Page of tier t (16-byte aligned fields, in this order):
- *    r[16] fp16 | vscale[16] fp16 | leaf rows [16][8*b_leaf]
- *    | upper rows [16][round_up_16(63*b_up/8)] | value rows [16][16*v_bits]
- *  Codes are packed LSB-first into one little-endian bit stream per token row
- *  (code i at bit i*b); int4 values put channel 2i in the low nibble (two's
- *  complement).  Pad bits are 0.  Slots of tokens never written keep whatever
- *  the caller put there (zero the pools to compare pages byte for byte).
+ *  Page of tier t, in this order (all fields 16-byte aligned):
+ *    r[16] fp16 | vscale[16] fp16 | code planes | value rows [16][16*v_bits]
+ *  Codes of a token are regrouped into 8 subtree blocks, block s for leaves
+ *  8s..8s+7: L[s][j] = leaf code 8s+j; U[s][0..3] = level-1 nodes 4s..4s+3,
+ *  U[s][4..5] = level-2 nodes 2s, 2s+1, U[s][6] = level-3 node s, U[s][7] =
+ *  top node s for s < 7 (top nodes: the 4 level-4 nodes, the 2 level-5
+ *  nodes, the root), U[7][7] = 0.  Code planes, each [16 tokens][8 blocks]
+ *  [width], little-endian:
+ *    T1: width 16: bytes 0..7 = L[s][0..7], bytes 8..15 = U[s][0..7];
+ *    T2: width 8: u32 nibble j = L[s][j], u32 nibble j = U[s][j] & 15;
+ *        width 2: u16 bits 2j..2j+1 = U[s][j] >> 4;
+ *    T3: width 4: u32 nibble j = U[s][j]; width 2: u16 bits 2j..2j+1 =
+ *        L[s][j] & 3; width 1: u8 bit j = L[s][j] >> 2.
+ *  Value row position p = 16g + 2m + h (g, m = 0..7, h = 0..1) holds channel
+ *  16m + g + 8h.  int8 (T1): token r has a 128-byte row whose 16-byte chunk g
+ *  (positions 16g..16g+15) is stored at chunk g ^ (r & 6).  int4 (T2, T3):
+ *  tokens 2i and 2i+1 share a 128-byte block; its 16-byte chunk g ^ (2i & 6)
+ *  holds chunk g (8 bytes, even position in the low nibble, two's
+ *  complement) of token 2i, then that of token 2i+1.  Unused bits are 0.  Slots of tokens never written keep
+ *  whatever the caller put there (zero the pools to compare pages byte for
+ *  byte).  This grouping gives each decode lane one aligned block per token
+ *  and each tensor-core thread its value fragments in contiguous,
+ *  bank-conflict-free 16-byte loads.
  *
  *  Page table: int32 [H_kv][total_pages].  Bits 31..30 = tier (0 drop, 1..3),
  *  bits 29..0 = page index inside that tier's pool.  Sequence b owns logical

@@ -76,16 +76,15 @@ static const int ORC_BLEAF[4] = {0, 8, 4, 3};
 static const int ORC_BUP[4] = {0, 8, 6, 4};
 static const int ORC_VBITS[4] = {0, 8, 4, 4};
 
-/* Byte sizes of one token row of each field in a page of the given tier. */
-static int leaf_row_bytes(int t) { return (ORC_D / 2) * ORC_BLEAF[t] / 8; }
-static int up_row_bytes(int t) { return ((ORC_D / 2 - 1) * ORC_BUP[t] + 127) / 128 * 16; }
+/* Bytes of the code blocks of one token (8 subtree blocks) and of one value
+ * row, per tier. */
+static int code_row_bytes(int t) { return t == 1 ? 128 : t == 2 ? 80 : 56; }
 static int v_row_bytes(int t) { return ORC_D * ORC_VBITS[t] / 8; }
 
-/* Field offsets inside a page: r[16] fp16, vscale[16] fp16, leaf rows, upper
- * rows, value rows. */
-static int off_leaf(int t) { (void)t; return 2 * ORC_PAGE * 2; }
-static int off_up(int t) { return off_leaf(t) + ORC_PAGE * leaf_row_bytes(t); }
-static int off_v(int t) { return off_up(t) + ORC_PAGE * up_row_bytes(t); }
+/* Field offsets inside a page: r[16] fp16, vscale[16] fp16, code planes,
+ * value rows. */
+static int off_codes(int t) { (void)t; return 2 * ORC_PAGE * 2; }
+static int off_v(int t) { return off_codes(t) + ORC_PAGE * code_row_bytes(t); }
 
 int orc_page_bytes(int t)
 {
@@ -326,63 +325,160 @@ void orc_attention(int64_t n_keys, int d, const double* khat, const double* vhat
 
 /* -------------------------------------------------------- page format -- */
 
-/* Write the low `bits` bits of `val` into a little-endian, LSB-first bit
- * stream starting at bit `pos` of `row`. */
-static void put_bits(uint8_t* row, int pos, int bits, unsigned val)
+/* The codes of one token regrouped into 8 subtree blocks, one per 8-leaf
+ * subtree s:  L[s][j] = leaf 8s+j;  U[s][0..3] = level-1 nodes 4s..4s+3,
+ * U[s][4..5] = level-2 nodes 2s, 2s+1, U[s][6] = level-3 node s, and
+ * U[s][7] = top node s for s < 7, where the top nodes are level 4 (4 nodes),
+ * level 5 (2 nodes) and the root; U[7][7] = 0.  Level-order index of level-1
+ * node m is m, level 2 is 32 + m, level 3 is 48 + m, level 4 is 56 + m,
+ * level 5 is 60 + m, the root 62. */
+static void to_blocks(const uint8_t* leaf, const uint8_t* up, uint8_t L[8][8], uint8_t U[8][8])
 {
-    for (int i = 0; i < bits; ++i) {
-        int p = pos + i;
-        if ((val >> i) & 1u) row[p >> 3] |= (uint8_t)(1u << (p & 7));
-        else row[p >> 3] &= (uint8_t)~(1u << (p & 7));
+    for (int s = 0; s < 8; ++s) {
+        for (int j = 0; j < 8; ++j) L[s][j] = leaf[8 * s + j];
+        for (int j = 0; j < 4; ++j) U[s][j] = up[4 * s + j];
+        U[s][4] = up[32 + 2 * s];
+        U[s][5] = up[32 + 2 * s + 1];
+        U[s][6] = up[48 + s];
+        U[s][7] = s < 7 ? up[56 + s] : 0;
     }
 }
 
-static unsigned get_bits(const uint8_t* row, int pos, int bits)
+static void from_blocks(uint8_t L[8][8], uint8_t U[8][8], uint8_t* leaf, uint8_t* up)
 {
-    unsigned v = 0;
-    for (int i = 0; i < bits; ++i) {
-        int p = pos + i;
-        v |= (unsigned)((row[p >> 3] >> (p & 7)) & 1u) << i;
+    for (int s = 0; s < 8; ++s) {
+        for (int j = 0; j < 8; ++j) leaf[8 * s + j] = L[s][j];
+        for (int j = 0; j < 4; ++j) up[4 * s + j] = U[s][j];
+        up[32 + 2 * s] = U[s][4];
+        up[32 + 2 * s + 1] = U[s][5];
+        up[48 + s] = U[s][6];
+        if (s < 7) up[56 + s] = U[s][7];
     }
+}
+
+/* Value row position p = 16g + 2m + h (g, m = 0..7, h = 0..1) holds channel
+ * 16m + g + 8h. */
+static int v_channel_at(int p) { return 16 * ((p >> 1) & 7) + (p >> 4) + 8 * (p & 1); }
+
+/* Byte of the value section that holds row position p (0..127) of token
+ * `slot`.  int8 (T1): rows of 128 bytes, 16-byte chunk g = p/16 of row r
+ * stored at chunk g ^ (r & 6).  int4 (T2, T3): tokens 2i and 2i+1 share a
+ * 128-byte block of eight 16-byte chunks; chunk g ^ (2i & 6) holds 8 bytes of
+ * token 2i then 8 bytes of token 2i+1 (positions 16g .. 16g+15, two per byte,
+ * even position in the low nibble). */
+static int v_byte_at(int t, int slot, int p)
+{
+    int g = p >> 4, j = p & 15;
+    if (ORC_VBITS[t] == 8) return off_v(t) + slot * 128 + 16 * (g ^ (slot & 6)) + j;
+    int i = slot >> 1;
+    return off_v(t) + i * 128 + 16 * (g ^ ((2 * i) & 6)) + 8 * (slot & 1) + (j >> 1);
+}
+
+static void put_le(uint8_t* dst, int nbytes, uint64_t v)
+{
+    for (int i = 0; i < nbytes; ++i) dst[i] = (uint8_t)(v >> (8 * i));
+}
+
+static uint64_t get_le(const uint8_t* src, int nbytes)
+{
+    uint64_t v = 0;
+    for (int i = 0; i < nbytes; ++i) v |= (uint64_t)src[i] << (8 * i);
     return v;
 }
 
 /* Store one token (d = 128) into slot `slot` of a page of tier t (1..3).
- * Pad bits of the rows are written as zero. */
+ * Code planes (each [16 tokens][8 blocks][width] bytes, in this order):
+ *   T1: width 16: bytes 0..7 = L[s][0..7], bytes 8..15 = U[s][0..7];
+ *   T2: width 8: u32 with nibble j = L[s][j], then u32 with nibble j =
+ *       U[s][j] & 15;  width 2: u16 with bits 2j..2j+1 = U[s][j] >> 4;
+ *   T3: width 4: u32 with nibble j = U[s][j];  width 2: u16 with bits
+ *       2j..2j+1 = L[s][j] & 3;  width 1: u8 with bit j = L[s][j] >> 2.
+ * Multi-byte fields are little-endian.  Value row position p holds channel
+ * v_channel_at(p), stored at v_byte_at (int4: two's complement nibbles). */
 void orc_pack_token(int t, int slot, const uint8_t* leaf, const uint8_t* up, uint16_t r16,
                     uint16_t s16, const int8_t* vq, uint8_t* page)
 {
-    int bl = ORC_BLEAF[t], bu = ORC_BUP[t], vb = ORC_VBITS[t];
-    page[2 * slot] = (uint8_t)(r16 & 0xff);
-    page[2 * slot + 1] = (uint8_t)(r16 >> 8);
-    page[2 * ORC_PAGE + 2 * slot] = (uint8_t)(s16 & 0xff);
-    page[2 * ORC_PAGE + 2 * slot + 1] = (uint8_t)(s16 >> 8);
-    uint8_t* lrow = page + off_leaf(t) + slot * leaf_row_bytes(t);
-    memset(lrow, 0, (size_t)leaf_row_bytes(t));
-    for (int j = 0; j < ORC_D / 2; ++j) put_bits(lrow, j * bl, bl, leaf[j]);
-    uint8_t* urow = page + off_up(t) + slot * up_row_bytes(t);
-    memset(urow, 0, (size_t)up_row_bytes(t));
-    for (int m = 0; m < ORC_D / 2 - 1; ++m) put_bits(urow, m * bu, bu, up[m]);
-    uint8_t* vrow = page + off_v(t) + slot * v_row_bytes(t);
-    memset(vrow, 0, (size_t)v_row_bytes(t));
-    for (int c = 0; c < ORC_D; ++c) put_bits(vrow, c * vb, vb, (unsigned)(vq[c] & ((1 << vb) - 1)));
+    uint8_t L[8][8], U[8][8];
+    to_blocks(leaf, up, L, U);
+    put_le(page + 2 * slot, 2, r16);
+    put_le(page + 2 * ORC_PAGE + 2 * slot, 2, s16);
+    uint8_t* c = page + off_codes(t);
+    for (int s = 0; s < 8; ++s) {
+        int blk = slot * 8 + s;
+        if (t == 1) {
+            for (int j = 0; j < 8; ++j) {
+                c[blk * 16 + j] = L[s][j];
+                c[blk * 16 + 8 + j] = U[s][j];
+            }
+        } else if (t == 2) {
+            uint64_t a = 0, b = 0;
+            for (int j = 0; j < 8; ++j) {
+                a |= (uint64_t)L[s][j] << (4 * j);
+                a |= (uint64_t)(U[s][j] & 15) << (32 + 4 * j);
+                b |= (uint64_t)(U[s][j] >> 4) << (2 * j);
+            }
+            put_le(c + blk * 8, 8, a);
+            put_le(c + ORC_PAGE * 8 * 8 + blk * 2, 2, b);
+        } else {
+            uint64_t a = 0, b = 0, e = 0;
+            for (int j = 0; j < 8; ++j) {
+                a |= (uint64_t)U[s][j] << (4 * j);
+                b |= (uint64_t)(L[s][j] & 3) << (2 * j);
+                e |= (uint64_t)(L[s][j] >> 2) << j;
+            }
+            put_le(c + blk * 4, 4, a);
+            put_le(c + ORC_PAGE * 8 * 4 + blk * 2, 2, b);
+            put_le(c + ORC_PAGE * 8 * 6 + blk, 1, e);
+        }
+    }
+    for (int p = 0; p < ORC_D; ++p) {
+        int code = vq[v_channel_at(p)];
+        int off = v_byte_at(t, slot, p);
+        if (ORC_VBITS[t] == 8) page[off] = (uint8_t)code;
+        else if (p & 1) page[off] = (uint8_t)((page[off] & 0x0f) | ((code & 15) << 4));
+        else page[off] = (uint8_t)((page[off] & 0xf0) | (code & 15));
+    }
 }
 
 void orc_unpack_token(int t, int slot, const uint8_t* page, uint8_t* leaf, uint8_t* up,
                       uint16_t* r16, uint16_t* s16, int8_t* vq)
 {
-    int bl = ORC_BLEAF[t], bu = ORC_BUP[t], vb = ORC_VBITS[t];
-    *r16 = (uint16_t)(page[2 * slot] | (page[2 * slot + 1] << 8));
-    *s16 = (uint16_t)(page[2 * ORC_PAGE + 2 * slot] | (page[2 * ORC_PAGE + 2 * slot + 1] << 8));
-    const uint8_t* lrow = page + off_leaf(t) + slot * leaf_row_bytes(t);
-    for (int j = 0; j < ORC_D / 2; ++j) leaf[j] = (uint8_t)get_bits(lrow, j * bl, bl);
-    const uint8_t* urow = page + off_up(t) + slot * up_row_bytes(t);
-    for (int m = 0; m < ORC_D / 2 - 1; ++m) up[m] = (uint8_t)get_bits(urow, m * bu, bu);
-    const uint8_t* vrow = page + off_v(t) + slot * v_row_bytes(t);
-    for (int c = 0; c < ORC_D; ++c) {
-        int raw = (int)get_bits(vrow, c * vb, vb);
-        if (raw >= (1 << (vb - 1))) raw -= (1 << vb); /* two's complement */
-        vq[c] = (int8_t)raw;
+    uint8_t L[8][8], U[8][8];
+    *r16 = (uint16_t)get_le(page + 2 * slot, 2);
+    *s16 = (uint16_t)get_le(page + 2 * ORC_PAGE + 2 * slot, 2);
+    const uint8_t* c = page + off_codes(t);
+    for (int s = 0; s < 8; ++s) {
+        int blk = slot * 8 + s;
+        if (t == 1) {
+            for (int j = 0; j < 8; ++j) {
+                L[s][j] = c[blk * 16 + j];
+                U[s][j] = c[blk * 16 + 8 + j];
+            }
+        } else if (t == 2) {
+            uint64_t a = get_le(c + blk * 8, 8), b = get_le(c + ORC_PAGE * 8 * 8 + blk * 2, 2);
+            for (int j = 0; j < 8; ++j) {
+                L[s][j] = (uint8_t)((a >> (4 * j)) & 15);
+                U[s][j] = (uint8_t)(((a >> (32 + 4 * j)) & 15) | (((b >> (2 * j)) & 3) << 4));
+            }
+        } else {
+            uint64_t a = get_le(c + blk * 4, 4), b = get_le(c + ORC_PAGE * 8 * 4 + blk * 2, 2),
+                     e = get_le(c + ORC_PAGE * 8 * 6 + blk, 1);
+            for (int j = 0; j < 8; ++j) {
+                U[s][j] = (uint8_t)((a >> (4 * j)) & 15);
+                L[s][j] = (uint8_t)(((b >> (2 * j)) & 3) | (((e >> j) & 1) << 2));
+            }
+        }
+    }
+    from_blocks(L, U, leaf, up);
+    for (int p = 0; p < ORC_D; ++p) {
+        int off = v_byte_at(t, slot, p);
+        int raw;
+        if (ORC_VBITS[t] == 8) raw = (int8_t)page[off];
+        else {
+            raw = (page[off] >> (4 * (p & 1))) & 15;
+            if (raw >= 8) raw -= 16; /* two's complement */
+        }
+        vq[v_channel_at(p)] = (int8_t)raw;
     }
 }
 

@@ -319,36 +319,64 @@ def test_page_layout_golden():
     g = json.load(open(os.path.join(GOLD, "page_layout.json")))
     for t in (1, 2, 3):
         assert oracle.page_bytes(t) == g["page_bytes"][str(t)]
-    z_up = np.zeros(63, np.uint8)
     z_v = np.zeros(128, np.int8)
-    # T3 leaf row of codes j mod 8
-    page = np.zeros(oracle.page_bytes(3), np.uint8)
-    leaf = (np.arange(64) % 8).astype(np.uint8)
-    oracle.pack_token(3, 0, leaf, z_up, 0, 0, z_v, page)
-    assert page[64:67].tolist() == g["t3_leaf_codes_j_mod_8_first_bytes"]
-    # T2 upper row of codes m
+    u32 = lambda b: int.from_bytes(bytes(b), "little")
+    # T1
+    page = np.zeros(oracle.page_bytes(1), np.uint8)
+    oracle.pack_token(1, 0, np.arange(64).astype(np.uint8), np.arange(63).astype(np.uint8), 0, 0, z_v, page)
+    assert page[64:80].tolist() == g["t1_block0"]
+    assert page[64 + 7 * 16:64 + 8 * 16].tolist() == g["t1_block7"]
+    assert page[64 + 6 * 16 + 15] == g["t1_block6_last"]
+    # T2
     page = np.zeros(oracle.page_bytes(2), np.uint8)
-    up = np.arange(63).astype(np.uint8)
-    oracle.pack_token(2, 0, np.zeros(64, np.uint8), up, 0, 0, z_v, page)
-    off_up = 64 + 16 * 32
-    assert page[off_up:off_up + 3].tolist() == g["t2_up_codes_m_first_bytes"]
-    assert page[off_up + 46:off_up + 48].tolist() == g["t2_up_codes_m_bytes_46_47"]
-    # int4 nibbles
-    for pair, want in g["int4_pairs"]:
-        if want is None:
-            continue
-        page = np.zeros(oracle.page_bytes(2), np.uint8)
-        vq = np.zeros(128, np.int8)
-        vq[0:2] = pair
-        oracle.pack_token(2, 0, np.zeros(64, np.uint8), z_up, 0, 0, vq, page)
-        off_v = 64 + 16 * 32 + 16 * 48
-        assert page[off_v] == want
+    oracle.pack_token(2, 0, (np.arange(64) % 16).astype(np.uint8), np.arange(63).astype(np.uint8), 0, 0,
+                      z_v, page)
+    assert [u32(page[64:68]), u32(page[68:72])] == g["t2_block0_words"]
+    assert u32(page[64 + 1024:64 + 1026]) == g["t2_block0_high"]
+    # T3
+    page = np.zeros(oracle.page_bytes(3), np.uint8)
+    oracle.pack_token(3, 0, (np.arange(64) % 8).astype(np.uint8), (np.arange(63) % 16).astype(np.uint8), 0,
+                      0, z_v, page)
+    assert u32(page[64:68]) == g["t3_block0_upper"]
+    assert u32(page[64 + 512:64 + 514]) == g["t3_block0_leaf_low"]
+    assert page[64 + 768] == g["t3_block0_leaf_high"]
+    # values
+    page = np.zeros(oracle.page_bytes(1), np.uint8)
+    oracle.pack_token(1, 0, np.zeros(64, np.uint8), np.zeros(63, np.uint8), 0, 0,
+                      (np.arange(128) - 64).astype(np.int8), page)
+    assert page[2112:2115].tolist() == g["v_int8_first_bytes"]
+    assert page[2112 + 16] == g["v_int8_byte16"]
+    page = np.zeros(oracle.page_bytes(1), np.uint8)
+    oracle.pack_token(1, 3, np.zeros(64, np.uint8), np.zeros(63, np.uint8), 0, 0,
+                      (np.arange(128) - 64).astype(np.int8), page)
+    at = g["v_int8_slot3_chunk0_at"]
+    assert page[at:at + 3].tolist() == g["v_int8_first_bytes"]
+    page = np.zeros(oracle.page_bytes(2), np.uint8)
+    oracle.pack_token(2, 0, np.zeros(64, np.uint8), np.zeros(63, np.uint8), 0, 0,
+                      ((np.arange(128) % 15) - 7).astype(np.int8), page)
+    assert page[1344:1346].tolist() == g["v_int4_first_bytes"]
+    page = np.zeros(oracle.page_bytes(2), np.uint8)
+    oracle.pack_token(2, 3, np.zeros(64, np.uint8), np.zeros(63, np.uint8), 0, 0,
+                      ((np.arange(128) % 15) - 7).astype(np.int8), page)
+    at = g["v_int4_slot3_first_bytes_at"]
+    assert page[at:at + 2].tolist() == g["v_int4_first_bytes"]
 
 
-def test_pack_unpack_roundtrip_and_independent_bitstream():
-    """Pin: pack/unpack round-trips for every tier and slot, and each packed
-    row equals the same codes assembled as one Python integer (bit i*b of the
-    row holds code i), other slots untouched and pad bits zero."""
+def _blocks(leaf, up):
+    """Subtree blocks written out from the level-order definition."""
+    L = [[int(leaf[8 * s + j]) for j in range(8)] for s in range(8)]
+    U = []
+    for s in range(8):
+        u = [int(up[4 * s + j]) for j in range(4)] + [int(up[32 + 2 * s]), int(up[33 + 2 * s]), int(up[48 + s])]
+        u.append(int(up[56 + s]) if s < 7 else 0)
+        U.append(u)
+    return L, U
+
+
+def test_pack_unpack_roundtrip_and_independent_layout():
+    """Pin: pack/unpack round-trips for every tier and slot, and every field
+    equals the same codes assembled independently as Python integers from the
+    layout description; other slots are untouched."""
     rng = np.random.default_rng(7)
     for t, (bl, bu, vb) in TIERS.items():
         page = np.zeros(oracle.page_bytes(t), np.uint8)
@@ -365,17 +393,32 @@ def test_pack_unpack_roundtrip_and_independent_bitstream():
             u = oracle.unpack_token(t, slot, page)
             assert np.array_equal(u["leaf"], leaf) and np.array_equal(u["up"], up)
             assert u["r16"] == r16 and u["s16"] == s16 and np.array_equal(u["vq"], vq)
-            lrow = 64 * bl // 8
-            urow = (63 * bu + 127) // 128 * 16
-            vrow = 128 * vb // 8
-            big = sum(int(c) << (i * bl) for i, c in enumerate(leaf))
-            assert bytes(page[64 + slot * lrow: 64 + (slot + 1) * lrow]) == big.to_bytes(lrow, "little")
-            big = sum(int(c) << (i * bu) for i, c in enumerate(up))
-            o = 64 + 16 * lrow
-            assert bytes(page[o + slot * urow: o + (slot + 1) * urow]) == big.to_bytes(urow, "little")
-            big = sum((int(c) & (2 ** vb - 1)) << (i * vb) for i, c in enumerate(vq))
-            o = 64 + 16 * lrow + 16 * urow
-            assert bytes(page[o + slot * vrow: o + (slot + 1) * vrow]) == big.to_bytes(vrow, "little")
+            L, U = _blocks(leaf, up)
+            rd = lambda off, n: int.from_bytes(bytes(page[off:off + n]), "little")
+            for s in range(8):
+                blk = slot * 8 + s
+                if t == 1:
+                    assert page[64 + 16 * blk:64 + 16 * blk + 16].tolist() == L[s] + U[s]
+                elif t == 2:
+                    assert rd(64 + 8 * blk, 4) == sum(L[s][j] << (4 * j) for j in range(8))
+                    assert rd(68 + 8 * blk, 4) == sum((U[s][j] & 15) << (4 * j) for j in range(8))
+                    assert rd(64 + 1024 + 2 * blk, 2) == sum((U[s][j] >> 4) << (2 * j) for j in range(8))
+                else:
+                    assert rd(64 + 4 * blk, 4) == sum(U[s][j] << (4 * j) for j in range(8))
+                    assert rd(64 + 512 + 2 * blk, 2) == sum((L[s][j] & 3) << (2 * j) for j in range(8))
+                    assert rd(64 + 768 + blk, 1) == sum((L[s][j] >> 2) << j for j in range(8))
+            voff = 64 + 16 * {1: 128, 2: 80, 3: 56}[t]
+            for p in range(128):
+                ch = 16 * ((p >> 1) & 7) + (p >> 4) + 8 * (p & 1)
+                gq, j = p // 16, p % 16
+                if vb == 8:
+                    at = voff + slot * 128 + 16 * (gq ^ (slot & 6)) + j
+                    assert int(page[at].astype(np.int8)) == vq[ch]
+                else:
+                    i = slot // 2
+                    at = voff + i * 128 + 16 * (gq ^ ((2 * i) & 6)) + 8 * (slot % 2) + j // 2
+                    nib = (int(page[at]) >> (4 * (p % 2))) & 15
+                    assert (nib - 16 if nib >= 8 else nib) == vq[ch]
             assert int(page[2 * slot]) | int(page[2 * slot + 1]) << 8 == r16
             assert int(page[32 + 2 * slot]) | int(page[33 + 2 * slot]) << 8 == s16
 
