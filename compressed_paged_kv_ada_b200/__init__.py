@@ -11,6 +11,7 @@ from ._lib import (  # noqa: F401
     make_cache,
     sphkv_build_page_table,
     sphkv_decode_attention,
+    sphkv_decode_attention_noalloc,
     sphkv_decode_workspace_bytes,
     sphkv_encode,
     sphkv_page_bytes,

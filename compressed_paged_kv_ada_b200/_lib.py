@@ -44,7 +44,7 @@ class sphkv_cache(ctypes.Structure):
 _lib = None
 _EXPORTS = ("sphkv_page_bytes", "sphkv_last_error", "sphkv_encode", "sphkv_rdr_workspace_bytes",
             "sphkv_rdr_assign", "sphkv_build_page_table", "sphkv_decode_workspace_bytes",
-            "sphkv_decode_attention")
+            "sphkv_decode_attention", "sphkv_decode_attention_noalloc")
 
 
 def lib() -> ctypes.CDLL:
@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.sphkv_decode_attention.restype = c.c_int
         L.sphkv_decode_attention.argtypes = [c.POINTER(sphkv_cache), c.c_int32, P, P, P, P, c.c_size_t,
                                              P, P]
+        L.sphkv_decode_attention_noalloc.restype = c.c_int
+        L.sphkv_decode_attention_noalloc.argtypes = [c.POINTER(sphkv_cache), c.c_int32, P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -170,3 +172,12 @@ def sphkv_decode_attention(cache: sphkv_cache, H_q: int, q: torch.Tensor, out: t
         ctypes.byref(cache), int(H_q), _ptr(q, torch.float32, "q"), _ptr(out, torch.float32, "out"),
         _ptr(lse, torch.float32, "lse"), _ptr(workspace, torch.uint8, "workspace"),
         int(workspace.numel()), _ptr(status, torch.int32, "status"), _stream(stream)))
+
+
+def sphkv_decode_attention_noalloc(cache: sphkv_cache, H_q: int, q: torch.Tensor, out: torch.Tensor,
+                                   lse: torch.Tensor, status: Optional[torch.Tensor] = None, stream=None):
+    """Decode attention with the library's static scratch instead of a
+    caller workspace, for callers that cannot allocate device memory."""
+    _check("sphkv_decode_attention_noalloc", lib().sphkv_decode_attention_noalloc(
+        ctypes.byref(cache), int(H_q), _ptr(q, torch.float32, "q"), _ptr(out, torch.float32, "out"),
+        _ptr(lse, torch.float32, "lse"), _ptr(status, torch.int32, "status"), _stream(stream)))

@@ -34,6 +34,8 @@
 //             accumulators).  Value codes are exact in f16; the weights p*scale
 //             are split into f16 hi + lo parts (two MMAs), keeping ~22 bits.
 //   merge  -- one CTA per unit whose pages were split over several CTAs.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace sphkv {
@@ -857,6 +859,122 @@ extern "C" sphkv_status sphkv_decode_attention(const sphkv_cache* c, int32_t H_q
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) {
         sphkv_set_error("sphkv_decode_attention: launch failed: %s", cudaGetErrorString(err));
+        return SPHKV_ERR_DEVICE;
+    }
+    return SPHKV_OK;
+}
+
+// ----------------------------------------------------- no-allocation variant --
+// Some callers cannot hand the library a device workspace: an engine that owns
+// every byte of device memory and forbids allocation once it has started, or a
+// latency-critical loop where a cudaMalloc (and the synchronisation it can
+// imply) is not acceptable.  sphkv_decode_attention_noalloc serves them: the
+// same plan / decode / merge kernels run with their scratch (unit page
+// offsets and split-KV partials) in the file-scope array below, which every
+// GPU that loads this library holds until the process exits.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;   // 4 MiB per device
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+}  // namespace
+
+extern "C" sphkv_status sphkv_decode_attention_noalloc(const sphkv_cache* c, int32_t H_q, const float* q,
+                                                       float* out, float* lse, int32_t* status_dev,
+                                                       void* stream)
+{
+    if (!c || !q || !out || !lse) {
+        sphkv_set_error("sphkv_decode_attention_noalloc: null argument");
+        return SPHKV_ERR_ARG;
+    }
+    if (c->B <= 0 || c->H_kv <= 0 || !c->page_offsets || !c->seq_lens || !c->page_table ||
+        c->total_pages < 0) {
+        sphkv_set_error("sphkv_decode_attention_noalloc: bad cache descriptor");
+        return SPHKV_ERR_ARG;
+    }
+    if (H_q != kG * c->H_kv) {
+        sphkv_set_error("sphkv_decode_attention_noalloc: H_q / H_kv must be %d (got H_q=%d, H_kv=%d)", kG,
+                        H_q, c->H_kv);
+        return SPHKV_ERR_ARG;
+    }
+    if ((uintptr_t)q & 15) {
+        sphkv_set_error("sphkv_decode_attention_noalloc: q must be 16-byte aligned");
+        return SPHKV_ERR_ARG;
+    }
+    if ((int64_t)c->H_kv * c->total_pages > 0x7fffffffLL || (int64_t)c->B * c->H_kv > (1 << 24)) {
+        sphkv_set_error("sphkv_decode_attention_noalloc: cache too large for 32-bit page indices");
+        return SPHKV_ERR_ARG;
+    }
+    DecodeParams p{};
+    for (int t = 1; t <= 3; ++t) {
+        p.pool[t] = c->pool[t - 1];
+        p.pool_pages[t] = c->pool[t - 1] ? c->pool_pages[t - 1] : 0;
+        if ((uintptr_t)c->pool[t - 1] & 15) {
+            sphkv_set_error("sphkv_decode_attention_noalloc: pool %d is not 16-byte aligned", t);
+            return SPHKV_ERR_ARG;
+        }
+    }
+    p.n_cta = pick_ctas(c->H_kv, c->total_pages, sm_count(0));
+    size_t part_off;
+    const size_t need = ws_layout(c->B, c->H_kv, p.n_cta, &part_off);
+    if (need > kNoAllocScratchBytes) {
+        sphkv_set_error(
+            "sphkv_decode_attention_noalloc: this cache needs %zu bytes of scratch but the static area holds "
+            "%zu; use sphkv_decode_attention with a caller workspace",
+            need, kNoAllocScratchBytes);
+        return SPHKV_ERR_ARG;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        sphkv_set_error("sphkv_decode_attention_noalloc: no usable current device");
+        return SPHKV_ERR_DEVICE;
+    }
+    void* scratch = nullptr;
+    {
+        // First call on each device: look up the device address of the static
+        // array with that device current (a host-side symbol is not a device
+        // address).  This first call should come before any stream capture.
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_addr[dev]) {
+            void* a = nullptr;
+            const cudaError_t e = cudaGetSymbolAddress(&a, g_noalloc_scratch);
+            if (e != cudaSuccess || !a) {
+                sphkv_set_error("sphkv_decode_attention_noalloc: cudaGetSymbolAddress failed: %s",
+                                cudaGetErrorString(e));
+                return SPHKV_ERR_DEVICE;
+            }
+            if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+                cudaSuccess) {
+                sphkv_set_error("sphkv_decode_attention_noalloc: cannot reserve %d bytes of shared memory",
+                                kSmemBytes);
+                return SPHKV_ERR_DEVICE;
+            }
+            g_noalloc_addr[dev] = a;
+        }
+        scratch = g_noalloc_addr[dev];
+    }
+    p.page_offsets = c->page_offsets;
+    p.seq_lens = c->seq_lens;
+    p.page_table = c->page_table;
+    p.total_pages = c->total_pages;
+    p.B = c->B;
+    p.H_kv = c->H_kv;
+    p.H_q = H_q;
+    p.n_units = c->B * c->H_kv;
+    p.q = q;
+    p.out = out;
+    p.lse = lse;
+    p.unit_start = (int32_t*)scratch;
+    p.partial = (float*)((uint8_t*)scratch + part_off);
+    p.status = status_dev;
+    cudaStream_t s = (cudaStream_t)stream;
+    plan_kernel<<<1, 1024, 0, s>>>(p);
+    decode_kernel<<<p.n_cta, kThreads, kSmemBytes, s>>>(p);
+    merge_kernel<<<p.n_units, kG * kD, 0, s>>>(p);
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) {
+        sphkv_set_error("sphkv_decode_attention_noalloc: launch failed: %s", cudaGetErrorString(err));
         return SPHKV_ERR_DEVICE;
     }
     return SPHKV_OK;

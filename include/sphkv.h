@@ -200,6 +200,30 @@ sphkv_status sphkv_decode_attention(const sphkv_cache* cache, int32_t H_q, const
                                     float* out, float* lse, void* workspace, size_t ws_bytes,
                                     int32_t* status_dev, void* stream);
 
+/*
+ * sphkv_decode_attention_noalloc -- sphkv_decode_attention without a caller
+ *   workspace.  The paper has no counterpart: this entry point exists for
+ *   callers that cannot allocate device memory, such as an engine that owns
+ *   every byte of device memory and forbids allocation after start-up, or a
+ *   latency-critical loop where cudaMalloc and the synchronisation it can
+ *   imply are not acceptable.  It allocates nothing: the decode scratch (unit
+ *   page offsets and split-KV partials) lives in a 4 MiB static device array
+ *   inside the library, which every GPU that loads the library holds until
+ *   the process exits.  Arguments, results and errors are those of
+ *   sphkv_decode_attention; q, out and lse are still the caller's.
+ *   - A cache whose scratch need (sphkv_decode_workspace_bytes with n_sm = 0)
+ *     exceeds 4 MiB is rejected with SPHKV_ERR_ARG and a message naming both
+ *     sizes; nothing is launched.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents (every value the kernels read is written earlier in the same
+ *     call, so nothing needs clearing).  Calls whose work overlaps on the GPU,
+ *     e.g. on two streams, race on it: serialise them.
+ */
+sphkv_status sphkv_decode_attention_noalloc(const sphkv_cache* cache, int32_t H_q, const float* q,
+                                            float* out, float* lse, int32_t* status_dev, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
