@@ -57,9 +57,23 @@ constexpr int kLutBytes = kLutT3 + 16 * kLutRow;
 constexpr int kStageOff = kLutBytes;
 constexpr int kPbufOff = kStageOff + kWarps * kStages * kStageBytes;
 constexpr int kPbufFloats = 16 * kG + 2 * kG;   // p*scale per (token, head); alpha per head; pad
-constexpr int kBarOff = kPbufOff + kWarps * kPbufFloats * 4;
+// Query-folded leaf tables of the current unit for T2 and T3: entry (code c,
+// leaf j = 8s + i) holds q_h[2j] cos(phi_c) + q_h[2j+1] sin(phi_c) for the 4
+// heads (16 bytes) at byte (c << 10) + 128 s + 16 (i ^ s): the 8 lanes of a
+// token look up the same i for different s, which lands in 8 distinct banks.
+constexpr int kFoldOff = kPbufOff + kWarps * kPbufFloats * 4;
+constexpr int kFoldT2 = 0, kFoldT3 = 16 * 1024;
+constexpr int kFoldBytes = kFoldT3 + 8 * 1024;
+// The unit's query for T1 leaves: even dims and odd dims of leaf j = 8s + i in
+// two arrays of 16-byte entries (4 heads) at entry 8s + ((i + s) & 7), so the 8
+// subtree lanes of a token read 8 distinct banks.
+constexpr int kQOff = kFoldOff + kFoldBytes;
+constexpr int kQBytes = 2 * kLeaves * 16;
+constexpr int kBarOff = kQOff + kQBytes;
 constexpr int kSmemBytes = kBarOff + kWarps * kStages * 8;
-static_assert(kStageOff % 128 == 0 && kPbufOff % 16 == 0 && kBarOff % 8 == 0, "smem alignment");
+static_assert(kStageOff % 128 == 0 && kPbufOff % 16 == 0 && kFoldOff % 128 == 0 && kQOff % 128 == 0 &&
+                  kBarOff % 8 == 0,
+              "smem alignment");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 // CTA merge scratch (aliases the stage ring): m[16][4], l[16][4], o[16][4][128]
 static_assert((2 * kWarps * kG + kWarps * kG * kD) * 4 <= kWarps * kStages * kStageBytes, "merge scratch");
@@ -225,11 +239,14 @@ struct WarpState {
     float acc[8][4];     // MMA accumulators: tile m = dims 16m..16m+15
 };
 
-// LUT byte offsets (tier base | code << 8 | replica << 3) of the 8 leaf and 8
-// upper codes of one subtree block.  base_rep = tier base | (lane & 15) << 3.
+// Offsets of the 8 leaf and 8 upper codes of one subtree block.  Upper codes
+// and T1 leaves: byte offset code << 8 | replica << 3 inside the tier's LUT,
+// with base_rep = (lane & 15) << 3.  T2/T3 leaves: offset into the
+// query-folded table, (code << 10 | 144 s) ^ 16 i for leaf i of subtree s,
+// with fold_lane = 144 s.
 template <int T>
-__device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uint32_t base_rep, uint32_t (&lo)[8],
-                                              uint32_t (&uo)[8])
+__device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uint32_t base_rep, uint32_t fold_lane,
+                                              uint32_t (&lo)[8], uint32_t (&uo)[8])
 {
     if (T == 1) {   // byte codes: one permute places the code in bits 8..15
         const uint4 w = *(const uint4*)(codes + blk * 16);
@@ -245,7 +262,7 @@ __device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uin
         const uint32_t h = *(const uint16_t*)(codes + kP * 64 + blk * 2);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            lo[j] = (((w.x >> (4 * j)) & 15u) << 8) | base_rep;
+            lo[j] = ((((w.x >> (4 * j)) & 15u) << 10) | fold_lane) ^ (16u * j);
             uo[j] = (((w.y >> (4 * j)) & 15u) << 8) | (((h >> (2 * j)) & 3u) << 12) | base_rep;
         }
     } else {
@@ -254,20 +271,18 @@ __device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uin
         const uint32_t l1 = codes[kP * 48 + blk];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            lo[j] = (((l2 >> (2 * j)) & 3u) << 8) | (((l1 >> j) & 1u) << 10) | base_rep;
+            lo[j] = ((((l2 >> (2 * j)) & 3u) << 10) | (((l1 >> j) & 1u) << 12) | fold_lane) ^ (16u * j);
             uo[j] = (((u >> (4 * j)) & 15u) << 8) | base_rep;
         }
     }
 }
 
-// (cos, sin) of a leaf or an upper code at LUT byte offset `off`.
-__device__ __forceinline__ float2 lut_leaf(const uint8_t* smem, uint32_t off)
+// 2^x on the special-function unit (max relative error about 2^-22); -inf -> 0.
+__device__ __forceinline__ float fast_exp2(float x)
 {
-    return *(const float2*)(smem + off);
-}
-__device__ __forceinline__ float2 lut_up(const uint8_t* smem, uint32_t off)
-{
-    return *(const float2*)(smem + 128 + off);
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // Two halves packed as f16x2: `lo` in the low half.
@@ -286,26 +301,28 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// One page of tier `tier` already staged in shared memory at `pg`.  Only the
-// code extraction and the value conversion depend on the tier; the tree, the
-// softmax and the MMAs are one copy of code for all tiers (a small kernel keeps
-// the instruction cache warm while warps interleave pages of different tiers).
-__device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int valid, const float (&qr)[kG][16],
-                                             const uint8_t* smem, float* pbuf, int lane, WarpState& st)
+// Logits of the 16 tokens of one page of tier T staged at `pg`, written in the
+// log2 domain to pbuf[t * kG + head] (-inf for slots past `valid`).  Lane
+// (k, s) evaluates subtree s of tokens 4 pass + k for all 4 heads.
+template <int T>
+__device__ __forceinline__ void page_logits(const uint8_t* pg, int valid, const uint8_t* smem, float* pbuf, int lane)
 {
     const unsigned full = 0xffffffffu;
     const int k = lane >> 3, s = lane & 7;
     const int head = (s & 1) * 2 + ((s >> 1) & 1);   // head held after the shuffle levels
-    const uint32_t base_rep = (uint32_t)(tier == 1 ? kLutT1 : tier == 2 ? kLutT2 : kLutT3) | ((uint32_t)(lane & 15) << 3);
+    constexpr int kBase = T == 1 ? kLutT1 : T == 2 ? kLutT2 : kLutT3;
+    constexpr int kFold = kFoldOff + (T == 3 ? kFoldT3 : kFoldT2);
+    const uint8_t* lut = smem + kBase;
+    const uint32_t rep = (uint32_t)(lane & 15) << 3;
+    const uint32_t fold_lane = 144u * (uint32_t)s;
+    const float4* qe = (const float4*)(smem + kQOff);   // q[2j] of the 4 heads
+    const float4* qo = qe + kLeaves;                     // q[2j + 1]
     const uint8_t* codes = pg + Tier<1>::f.off_codes;
-    float lg0 = -INFINITY, lg1 = -INFINITY, lg2 = -INFINITY, lg3 = -INFINITY;
-#pragma unroll 1
+#pragma unroll 2
     for (int pass = 0; pass < 4; ++pass) {
         const int t = pass * 4 + k;
         uint32_t lo[8], uo[8];
-        if (tier == 1) block_offsets<1>(codes, t * 8 + s, base_rep, lo, uo);
-        else if (tier == 2) block_offsets<2>(codes, t * 8 + s, base_rep, lo, uo);
-        else block_offsets<3>(codes, t * 8 + s, base_rep, lo, uo);
+        block_offsets<T>(codes, t * 8 + s, rep, fold_lane, lo, uo);
         // top codes: block i carries top node i (level 4 nodes 0..3, level 5
         // nodes 0..1, root); lane s needs nodes s>>1, 4 + (s>>2) and 6
         const uint32_t o4 = __shfl_sync(full, uo[7], (lane & ~7) | (s >> 1));
@@ -315,26 +332,40 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
         float S1[4][kG];
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-            const float2 fa = lut_leaf(smem, lo[2 * m]);
-            const float2 fb = lut_leaf(smem, lo[2 * m + 1]);
-            const float2 fu = lut_up(smem, uo[m]);
-#pragma unroll
-            for (int h = 0; h < kG; ++h) {
-                const float L = fmaf(qr[h][4 * m + 1], fa.y, qr[h][4 * m] * fa.x);
-                const float R = fmaf(qr[h][4 * m + 3], fb.y, qr[h][4 * m + 2] * fb.x);
-                S1[m][h] = fmaf(fu.y, R, fu.x * L);
+            float L[kG], R[kG];
+            if (T == 1) {
+                const float2 fa = *(const float2*)(lut + lo[2 * m]);
+                const float2 fb = *(const float2*)(lut + lo[2 * m + 1]);
+                const int ea = 8 * s + ((2 * m + s) & 7), eb = 8 * s + ((2 * m + 1 + s) & 7);
+                const float4 ae = qe[ea], ao = qo[ea], be = qe[eb], bo = qo[eb];
+                L[0] = fmaf(ao.x, fa.y, ae.x * fa.x);
+                L[1] = fmaf(ao.y, fa.y, ae.y * fa.x);
+                L[2] = fmaf(ao.z, fa.y, ae.z * fa.x);
+                L[3] = fmaf(ao.w, fa.y, ae.w * fa.x);
+                R[0] = fmaf(bo.x, fb.y, be.x * fb.x);
+                R[1] = fmaf(bo.y, fb.y, be.y * fb.x);
+                R[2] = fmaf(bo.z, fb.y, be.z * fb.x);
+                R[3] = fmaf(bo.w, fb.y, be.w * fb.x);
+            } else {   // leaf terms already folded with the query
+                const float4 a = *(const float4*)(smem + kFold + lo[2 * m]);
+                const float4 c = *(const float4*)(smem + kFold + lo[2 * m + 1]);
+                L[0] = a.x; L[1] = a.y; L[2] = a.z; L[3] = a.w;
+                R[0] = c.x; R[1] = c.y; R[2] = c.z; R[3] = c.w;
             }
+            const float2 fu = *(const float2*)(lut + 128 + uo[m]);
+#pragma unroll
+            for (int h = 0; h < kG; ++h) S1[m][h] = fmaf(fu.y, R[h], fu.x * L[h]);
         }
         float S2[2][kG];
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
-            const float2 fu = lut_up(smem, uo[4 + n]);
+            const float2 fu = *(const float2*)(lut + 128 + uo[4 + n]);
 #pragma unroll
             for (int h = 0; h < kG; ++h) S2[n][h] = fmaf(fu.y, S1[2 * n + 1][h], fu.x * S1[2 * n][h]);
         }
         float S3[kG];
         {
-            const float2 fu = lut_up(smem, uo[6]);
+            const float2 fu = *(const float2*)(lut + 128 + uo[6]);
 #pragma unroll
             for (int h = 0; h < kG; ++h) S3[h] = fmaf(fu.y, S2[1][h], fu.x * S2[0][h]);
         }
@@ -344,7 +375,7 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
         const float r1 = __shfl_xor_sync(full, odd ? S3[1] : S3[3], 1);
         float T0, T1;
         {
-            const float2 fu = lut_up(smem, o4);
+            const float2 fu = *(const float2*)(lut + 128 + o4);
             T0 = fmaf(fu.y, odd ? S3[2] : r0, fu.x * (odd ? r0 : S3[0]));
             T1 = fmaf(fu.y, odd ? S3[3] : r1, fu.x * (odd ? r1 : S3[1]));
         }
@@ -353,7 +384,7 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
         const float r2 = __shfl_xor_sync(full, hi1 ? T0 : T1, 2);
         float U;
         {
-            const float2 fu = lut_up(smem, o5);
+            const float2 fu = *(const float2*)(lut + 128 + o5);
             U = fmaf(fu.y, hi1 ? T1 : r2, fu.x * (hi1 ? r2 : T0));
         }
         // root: lanes s, s^4 (both end with the same value)
@@ -361,29 +392,43 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
         const float r3 = __shfl_xor_sync(full, U, 4);
         float S;
         {
-            const float2 fu = lut_up(smem, o6);
+            const float2 fu = *(const float2*)(lut + 128 + o6);
             S = fmaf(fu.y, right ? U : r3, fu.x * (right ? r3 : U));
         }
         const float rr = __half2float(((const __half*)pg)[t]);
-        const float lv = t < valid ? rr * S * kLogitScale : -INFINITY;
-        lg0 = pass == 0 ? lv : lg0;
-        lg1 = pass == 1 ? lv : lg1;
-        lg2 = pass == 2 ? lv : lg2;
-        lg3 = pass == 3 ? lv : lg3;
+        if (s < 4) pbuf[t * kG + head] = t < valid ? rr * S * kLogitScale : -INFINITY;
     }
-    const float lg[4] = {lg0, lg1, lg2, lg3};
+}
+
+// One page of tier `tier` already staged in shared memory at `pg`.  The logits
+// are tier-specialised; the softmax and the value MMAs are one copy of code
+// for all tiers apart from the value conversion.
+__device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int valid, const uint8_t* smem, float* pbuf,
+                                             int lane, WarpState& st)
+{
+    const unsigned full = 0xffffffffu;
+    const int k = lane >> 3, s = lane & 7;
+    const int head = (s & 1) * 2 + ((s >> 1) & 1);
+    if (tier == 1) page_logits<1>(pg, valid, smem, pbuf, lane);
+    else if (tier == 2) page_logits<2>(pg, valid, smem, pbuf, lane);
+    else page_logits<3>(pg, valid, smem, pbuf, lane);
+    __syncwarp();
+    float lg[4];
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) lg[pass] = pbuf[(pass * 4 + k) * kG + head];
+    __syncwarp();
     // online softmax for this lane's head (lanes k = 0..3 share it)
     float pm = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
     pm = fmaxf(pm, __shfl_xor_sync(full, pm, 8));
     pm = fmaxf(pm, __shfl_xor_sync(full, pm, 16));
     const float m_new = fmaxf(st.m, pm);
-    const float alpha = exp2f(st.m - m_new);   // st.m = -inf on the first page -> 0
+    const float alpha = fast_exp2(st.m - m_new);   // st.m = -inf on the first page -> 0
     st.m = m_new;
     float psum = 0.f;
     const __half* vs = (const __half*)(pg + 2 * kP);
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
-        const float pv = exp2f(lg[pass] - m_new);
+        const float pv = fast_exp2(lg[pass] - m_new);
         psum += pv;
         const int t = pass * 4 + k;   // slots past `valid` may hold stale scales: weight exactly 0
         if (s < 4) pbuf[t * kG + head] = t < valid ? pv * __half2float(vs[t]) * kPScale : 0.f;
@@ -396,7 +441,7 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
     // rows = tokens 2c, 2c+1 (b0) and 2c+8, 2c+9 (b1); accumulator columns =
     // heads 2c, 2c+1.
     const int g = lane >> 2, c = lane & 3;
-    {
+    if (__any_sync(full, alpha != 1.f)) {   // a running max moved: rescale (rare after the first pages)
         const float2 al = *(const float2*)(pbuf + 16 * kG + 2 * (c & 1));
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
@@ -435,15 +480,15 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
             const int wi = m >> 1, b = 2 * (m & 1);   // byte b (h = 0) and b + 1 (h = 1) of word wi
-            // result byte 0 <- low token's byte, byte 2 <- high token's byte;
-            // | 0x6400 makes f16 1024 + u, u = code + 128
-            const uint32_t sel0 = (uint32_t)(b | ((4 + b) << 8));
-            const uint32_t sel1 = (uint32_t)((b + 1) | ((5 + b) << 8));
+            // interleave the two tokens' bytes b, b+1, then put 0x64 above each
+            // byte: f16 1024 + u with u = code + 128
+            const uint32_t sel = (uint32_t)(b | ((4 + b) << 4) | ((b + 1) << 8) | ((5 + b) << 12));
+            const uint32_t xy = __byte_perm(xs[wi], ys[wi], sel), zw = __byte_perm(zs[wi], ws[wi], sel);
             uint32_t a[4];
-            a[0] = (__byte_perm(xs[wi], ys[wi], sel0) & 0x00FF00FFu) | 0x64006400u;
-            a[1] = (__byte_perm(xs[wi], ys[wi], sel1) & 0x00FF00FFu) | 0x64006400u;
-            a[2] = (__byte_perm(zs[wi], ws[wi], sel0) & 0x00FF00FFu) | 0x64006400u;
-            a[3] = (__byte_perm(zs[wi], ws[wi], sel1) & 0x00FF00FFu) | 0x64006400u;
+            a[0] = __byte_perm(xy, 0x64646464u, 0x5140);
+            a[1] = __byte_perm(xy, 0x64646464u, 0x5342);
+            a[2] = __byte_perm(zw, 0x64646464u, 0x5140);
+            a[3] = __byte_perm(zw, 0x64646464u, 0x5342);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 __half2 hv = __hadd2(*(const __half2*)&a[i], bias);
@@ -547,24 +592,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
         const int len = p.seq_lens[b];
         const int32_t* ptab = p.page_table + (int64_t)g * p.total_pages + first;
 
-        // this lane's query slice: dims 16s .. 16s+15 of heads 4g .. 4g+3, as
-        // pairs of heads {4g + 2hp, 4g + 2hp + 1}
-        float qr[kG][16];
-        {
-            const int s = lane & 7;
+        // query-folded T2/T3 leaf tables for this unit (the previous segment
+        // ended with a barrier, so no warp still reads the old ones)
+        for (int e = tid; e < (16 + 8) * kLeaves; e += kThreads) {
+            const bool t3 = e >= 16 * kLeaves;
+            const int code = t3 ? (e - 16 * kLeaves) >> 6 : e >> 6, j = e & 63;
+            const float2 cs = *(const float2*)(smem + (t3 ? kLutT3 : kLutT2) + code * kLutRow);
+            float v[kG];
 #pragma unroll
             for (int h = 0; h < kG; ++h) {
-                const float4* src = (const float4*)(p.q + ((int64_t)b * p.H_q + g * kG + h) * kD + 16 * s);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float4 v = src[i];
-                    qr[h][4 * i] = v.x;
-                    qr[h][4 * i + 1] = v.y;
-                    qr[h][4 * i + 2] = v.z;
-                    qr[h][4 * i + 3] = v.w;
-                }
+                const float* qh = p.q + ((int64_t)b * p.H_q + g * kG + h) * kD;
+                v[h] = fmaf(qh[2 * j + 1], cs.y, qh[2 * j] * cs.x);
             }
+            const uint32_t off = ((uint32_t)code << 10) + 128u * (j >> 3) + 16u * ((j & 7) ^ (j >> 3));
+            *(float4*)(smem + kFoldOff + (t3 ? kFoldT3 : kFoldT2) + off) = make_float4(v[0], v[1], v[2], v[3]);
         }
+        for (int e = tid; e < 2 * kLeaves; e += kThreads) {   // q for T1 leaves
+            const int odd = e >= kLeaves, j = e & 63, sj = j >> 3, ij = j & 7;
+            float v[kG];
+#pragma unroll
+            for (int h = 0; h < kG; ++h) v[h] = p.q[((int64_t)b * p.H_q + g * kG + h) * kD + 2 * j + odd];
+            ((float4*)(smem + kQOff))[odd * kLeaves + 8 * sj + ((ij + sj) & 7)] = make_float4(v[0], v[1], v[2], v[3]);
+        }
+        __syncthreads();
         WarpState st;
         st.m = -INFINITY;
         st.l = 0.f;
@@ -637,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
             const uint8_t* pg = stage + cur * kStageBytes;
             const int valid = min(kP, len - lp_cur * kP);
             const int t = entry_tier(e_cur);
-            process_page(pg, t, valid, qr, smem, pbuf, lane, st);
+            process_page(pg, t, valid, smem, pbuf, lane, st);
             cur ^= 1;
             lp_cur = lp_nxt;
             e_cur = e_nxt;
