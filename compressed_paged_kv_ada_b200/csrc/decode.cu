@@ -13,22 +13,24 @@
 //
 // Launch structure (three kernels on the caller's stream):
 //   plan   -- 1 CTA: unit_start[u] = pages before unit u = (b, g), u = b*H_kv+g.
-//   decode -- persistent, one 384-thread CTA per SM.  The flattened page range
+//   decode -- persistent, one 512-thread CTA per SM.  The flattened page range
 //             [0, P) is cut into n_cta equal pieces; a CTA walks the units its
-//             piece overlaps.  Its 12 warps take the unit's pages round robin;
+//             piece overlaps.  Its 16 warps take the unit's pages round robin;
 //             each warp bulk-copies a page (cp.async.bulk, mbarrier completion)
 //             into a 2-stage ring in shared memory while it computes the
 //             previous one.
 //             Logits: 4 tokens per pass, 8 lanes per token; lane s owns the
 //             8-leaf subtree s (one aligned code block) and all 4 query heads,
-//             so each cos/sin lookup serves 4 heads.  The three top tree levels
-//             use shuffles that leave each lane a different head.  Tables sit in
-//             shared memory as rows of 256 bytes per code: 16 lane replicas of
-//             (cos, sin) for the leaf grid and for the upper grid, so a half
-//             warp's 64-bit lookups never share a bank and the address is one
-//             byte permute.  (Packed f32x2 arithmetic would need {cos,cos} and
-//             {sin,sin} pairs, i.e. 16-byte lookups; measured on B200 that
-//             doubles shared-memory traffic and is slower.)
+//             so each table lookup serves 4 heads.  The three top tree levels
+//             use shuffles that leave each lane a different head.  Cos/sin
+//             tables sit in shared memory with 16 lane replicas per code, so a
+//             half warp's 64-bit lookups never share a bank.  T2/T3 leaves
+//             (16 and 8 codes) instead index per-unit tables that already hold
+//             q[2j] cos(phi) + q[2j+1] sin(phi) for the 4 heads: one 16-byte
+//             lookup and no arithmetic per leaf.  (Packed f32x2 arithmetic in
+//             the upper levels would need {cos,cos} and {sin,sin} pairs, i.e.
+//             16-byte lookups; measured on B200 that doubles shared-memory
+//             traffic and is slower.)
 //             Values: out^T[dims x heads] += V^T[dims x 16 tokens] P^T[16 x 4]
 //             on the tensor cores (mma.sync m16n8k16, f16 operands, fp32
 //             accumulators).  Value codes are exact in f16; the weights p*scale
@@ -42,28 +44,34 @@ namespace sphkv {
 namespace {
 
 constexpr int kG = 4;               // query heads per kv head
-constexpr int kWarps = 12;
+constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 2;
 constexpr int kStageBytes = Tier<1>::f.page_bytes;  // largest page
 constexpr int kMinPagesPerCta = 64;
 constexpr int kPartStride = 132;    // floats per (slot, head): m, l, pad, pad, o[128]
 
-// LUT: per tier, one 256-byte row per code: [leaf (cos,sin) x 16 replicas]
-// [upper (cos,sin) x 16 replicas].  Rows: T1 256, T2 64, T3 16.
-constexpr int kLutRow = 256;
-constexpr int kLutT1 = 0, kLutT2 = 256 * kLutRow, kLutT3 = kLutT2 + 64 * kLutRow;
-constexpr int kLutBytes = kLutT3 + 16 * kLutRow;
+// Cos/sin tables.  T1: one 256-byte row per code, [leaf (cos,sin) x 16 lane
+// replicas][upper (cos,sin) x 16 replicas].  T2, T3: upper grid only, one
+// 128-byte row of 16 replicas per code (their leaves are read from the
+// query-folded table below), and one unreplicated (cos,sin) per T2 leaf code
+// for building it.
+constexpr int kLutT1 = 0;                    // 256 rows x 256 B
+constexpr int kLutT2 = 256 * 256;            // 64 rows x 128 B
+constexpr int kLutT3 = kLutT2 + 64 * 128;    // 16 rows x 128 B
+constexpr int kLeafT2 = kLutT3 + 16 * 128;   // 16 x (cos, sin)
+constexpr int kLutBytes = (kLeafT2 + 16 * 8 + 127) / 128 * 128;
 constexpr int kStageOff = kLutBytes;
 constexpr int kPbufOff = kStageOff + kWarps * kStages * kStageBytes;
 constexpr int kPbufFloats = 16 * kG + 2 * kG;   // p*scale per (token, head); alpha per head; pad
-// Query-folded leaf tables of the current unit for T2 and T3: entry (code c,
-// leaf j = 8s + i) holds q_h[2j] cos(phi_c) + q_h[2j+1] sin(phi_c) for the 4
-// heads (16 bytes) at byte (c << 10) + 128 s + 16 (i ^ s): the 8 lanes of a
-// token look up the same i for different s, which lands in 8 distinct banks.
-constexpr int kFoldOff = kPbufOff + kWarps * kPbufFloats * 4;
-constexpr int kFoldT2 = 0, kFoldT3 = 16 * 1024;
-constexpr int kFoldBytes = kFoldT3 + 8 * 1024;
+// Query-folded leaf table of the current unit on the T2 leaf grid (16 codes):
+// entry (code c, leaf j = 8s + i) holds q_h[2j] cos(phi_c) + q_h[2j+1]
+// sin(phi_c) for the 4 heads (16 bytes) at byte (c << 10) + 128 s + 16 (i ^ s):
+// the 8 lanes of a token look up the same i for different s, which lands in 8
+// distinct banks.  The T3 leaf grid (8 codes) is the even half of it: T3 code
+// c has the angle of T2 code 2c.
+constexpr int kFoldOff = (kPbufOff + kWarps * kPbufFloats * 4 + 127) / 128 * 128;
+constexpr int kFoldBytes = 16 * 1024;
 // The unit's query for T1 leaves: even dims and odd dims of leaf j = 8s + i in
 // two arrays of 16-byte entries (4 heads) at entry 8s + ((i + s) & 7), so the 8
 // subtree lanes of a token read 8 distinct banks.
@@ -239,9 +247,10 @@ struct WarpState {
     float acc[8][4];     // MMA accumulators: tile m = dims 16m..16m+15
 };
 
-// Offsets of the 8 leaf and 8 upper codes of one subtree block.  Upper codes
-// and T1 leaves: byte offset code << 8 | replica << 3 inside the tier's LUT,
-// with base_rep = (lane & 15) << 3.  T2/T3 leaves: offset into the
+// Offsets of the 8 leaf and 8 upper codes of one subtree block.  T1: byte
+// offset code << 8 | replica << 3 into its 256-byte rows; T2/T3 upper codes:
+// code << 7 | replica << 3; base_rep = (lane & 15) << 3.  T2/T3 leaves: offset
+// (T3 code c read as T2 code 2c) into the
 // query-folded table, (code << 10 | 144 s) ^ 16 i for leaf i of subtree s,
 // with fold_lane = 144 s.
 template <int T>
@@ -263,7 +272,7 @@ __device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uin
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             lo[j] = ((((w.x >> (4 * j)) & 15u) << 10) | fold_lane) ^ (16u * j);
-            uo[j] = (((w.y >> (4 * j)) & 15u) << 8) | (((h >> (2 * j)) & 3u) << 12) | base_rep;
+            uo[j] = (((w.y >> (4 * j)) & 15u) << 7) | (((h >> (2 * j)) & 3u) << 11) | base_rep;
         }
     } else {
         const uint32_t u = *(const uint32_t*)(codes + blk * 4);
@@ -271,8 +280,8 @@ __device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uin
         const uint32_t l1 = codes[kP * 48 + blk];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            lo[j] = ((((l2 >> (2 * j)) & 3u) << 10) | (((l1 >> j) & 1u) << 12) | fold_lane) ^ (16u * j);
-            uo[j] = (((u >> (4 * j)) & 15u) << 8) | base_rep;
+            lo[j] = ((((l2 >> (2 * j)) & 3u) << 11) | (((l1 >> j) & 1u) << 13) | fold_lane) ^ (16u * j);
+            uo[j] = (((u >> (4 * j)) & 15u) << 7) | base_rep;
         }
     }
 }
@@ -303,100 +312,90 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 
 // Logits of the 16 tokens of one page of tier T staged at `pg`, written in the
 // log2 domain to pbuf[t * kG + head] (-inf for slots past `valid`).  Lane
-// (k, s) evaluates subtree s of tokens 4 pass + k for all 4 heads.
+// (k, s) handles subtree s of tokens 4 pass + k for all 4 heads, top down:
+// the tree's value r S_root is the sum over leaves of (product of the factors
+// on the leaf's path: cos(psi) into a left child, sin(psi) into a right one)
+// times the leaf term q[2j] cos(phi_j) + q[2j+1] sin(phi_j).  The path
+// products do not depend on the head, so the per-head work is one
+// multiply-add per leaf (T2/T3, whose leaf terms are read from the
+// query-folded tables) or per dimension (T1).
 template <int T>
 __device__ __forceinline__ void page_logits(const uint8_t* pg, int valid, const uint8_t* smem, float* pbuf, int lane)
 {
     const unsigned full = 0xffffffffu;
     const int k = lane >> 3, s = lane & 7;
-    const int head = (s & 1) * 2 + ((s >> 1) & 1);   // head held after the shuffle levels
     constexpr int kBase = T == 1 ? kLutT1 : T == 2 ? kLutT2 : kLutT3;
-    constexpr int kFold = kFoldOff + (T == 3 ? kFoldT3 : kFoldT2);
+    constexpr int kUp = T == 1 ? 128 : 0;   // upper (cos, sin) inside a row
+    constexpr int kFold = kFoldOff;
     const uint8_t* lut = smem + kBase;
+    const uint8_t* lut_up = lut + kUp;
     const uint32_t rep = (uint32_t)(lane & 15) << 3;
     const uint32_t fold_lane = 144u * (uint32_t)s;
     const float4* qe = (const float4*)(smem + kQOff);   // q[2j] of the 4 heads
     const float4* qo = qe + kLeaves;                     // q[2j + 1]
     const uint8_t* codes = pg + Tier<1>::f.off_codes;
+    // ancestors of subtree s: level-4 node s>>1, level-5 node s>>2, the root;
+    // the subtree lies on their right (sin, byte 4 of the entry) or left side
+    const uint32_t side4 = (uint32_t)(s & 1) << 2, side5 = (uint32_t)((s >> 1) & 1) << 2;
+    const uint32_t side6 = (uint32_t)((s >> 2) & 1) << 2;
+    const bool b2 = (s >> 2) & 1, b1 = (s >> 1) & 1;
 #pragma unroll 2
     for (int pass = 0; pass < 4; ++pass) {
         const int t = pass * 4 + k;
         uint32_t lo[8], uo[8];
         block_offsets<T>(codes, t * 8 + s, rep, fold_lane, lo, uo);
         // top codes: block i carries top node i (level 4 nodes 0..3, level 5
-        // nodes 0..1, root); lane s needs nodes s>>1, 4 + (s>>2) and 6
+        // nodes 0..1, root)
         const uint32_t o4 = __shfl_sync(full, uo[7], (lane & ~7) | (s >> 1));
         const uint32_t o5 = __shfl_sync(full, uo[7], (lane & ~7) | (4 + (s >> 2)));
         const uint32_t o6 = __shfl_sync(full, uo[7], (lane & ~7) | 6);
-        // subtree of 8 leaves, 4 heads
-        float S1[4][kG];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            float L[kG], R[kG];
-            if (T == 1) {
-                const float2 fa = *(const float2*)(lut + lo[2 * m]);
-                const float2 fb = *(const float2*)(lut + lo[2 * m + 1]);
-                const int ea = 8 * s + ((2 * m + s) & 7), eb = 8 * s + ((2 * m + 1 + s) & 7);
-                const float4 ae = qe[ea], ao = qo[ea], be = qe[eb], bo = qo[eb];
-                L[0] = fmaf(ao.x, fa.y, ae.x * fa.x);
-                L[1] = fmaf(ao.y, fa.y, ae.y * fa.x);
-                L[2] = fmaf(ao.z, fa.y, ae.z * fa.x);
-                L[3] = fmaf(ao.w, fa.y, ae.w * fa.x);
-                R[0] = fmaf(bo.x, fb.y, be.x * fb.x);
-                R[1] = fmaf(bo.y, fb.y, be.y * fb.x);
-                R[2] = fmaf(bo.z, fb.y, be.z * fb.x);
-                R[3] = fmaf(bo.w, fb.y, be.w * fb.x);
-            } else {   // leaf terms already folded with the query
-                const float4 a = *(const float4*)(smem + kFold + lo[2 * m]);
-                const float4 c = *(const float4*)(smem + kFold + lo[2 * m + 1]);
-                L[0] = a.x; L[1] = a.y; L[2] = a.z; L[3] = a.w;
-                R[0] = c.x; R[1] = c.y; R[2] = c.z; R[3] = c.w;
-            }
-            const float2 fu = *(const float2*)(lut + 128 + uo[m]);
-#pragma unroll
-            for (int h = 0; h < kG; ++h) S1[m][h] = fmaf(fu.y, R[h], fu.x * L[h]);
+        float v = __half2float(((const __half*)pg)[t]) * kLogitScale;
+        v *= *(const float*)(lut_up + o6 + side6);
+        v *= *(const float*)(lut_up + o5 + side5);
+        v *= *(const float*)(lut_up + o4 + side4);
+        // level 3 (subtree root, code 6), level 2 (codes 4, 5), level 1 (codes 0..3)
+        float w2[2], w1[4], wl[8];
+        {
+            const float2 f = *(const float2*)(lut_up + uo[6]);
+            w2[0] = v * f.x;
+            w2[1] = v * f.y;
         }
-        float S2[2][kG];
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
-            const float2 fu = *(const float2*)(lut + 128 + uo[4 + n]);
+            const float2 f = *(const float2*)(lut_up + uo[4 + n]);
+            w1[2 * n] = w2[n] * f.x;
+            w1[2 * n + 1] = w2[n] * f.y;
+        }
 #pragma unroll
-            for (int h = 0; h < kG; ++h) S2[n][h] = fmaf(fu.y, S1[2 * n + 1][h], fu.x * S1[2 * n][h]);
+        for (int m = 0; m < 4; ++m) {
+            const float2 f = *(const float2*)(lut_up + uo[m]);
+            wl[2 * m] = w1[m] * f.x;
+            wl[2 * m + 1] = w1[m] * f.y;
         }
-        float S3[kG];
-        {
-            const float2 fu = *(const float2*)(lut + 128 + uo[6]);
+        float acc[kG];
 #pragma unroll
-            for (int h = 0; h < kG; ++h) S3[h] = fmaf(fu.y, S2[1][h], fu.x * S2[0][h]);
+        for (int j = 0; j < 8; ++j) {
+            if (T == 1) {
+                const float2 f = *(const float2*)(lut + lo[j]);
+                const float kx = wl[j] * f.x, ky = wl[j] * f.y;
+                const int e = 8 * s + ((j + s) & 7);
+                const float4 ev = qe[e], od = qo[e];
+                const float qev[kG] = {ev.x, ev.y, ev.z, ev.w}, qod[kG] = {od.x, od.y, od.z, od.w};
+#pragma unroll
+                for (int h = 0; h < kG; ++h) acc[h] = fmaf(qod[h], ky, j == 0 ? qev[h] * kx : fmaf(qev[h], kx, acc[h]));
+            } else {   // leaf terms already folded with the query
+                const float4 F = *(const float4*)(smem + kFold + lo[j]);
+                const float fv[kG] = {F.x, F.y, F.z, F.w};
+#pragma unroll
+                for (int h = 0; h < kG; ++h) acc[h] = j == 0 ? wl[j] * fv[h] : fmaf(wl[j], fv[h], acc[h]);
+            }
         }
-        // level 4: lanes s, s^1 hold sibling subtrees; even lane keeps heads 0,1
-        const bool odd = s & 1;
-        const float r0 = __shfl_xor_sync(full, odd ? S3[0] : S3[2], 1);
-        const float r1 = __shfl_xor_sync(full, odd ? S3[1] : S3[3], 1);
-        float T0, T1;
-        {
-            const float2 fu = *(const float2*)(lut + 128 + o4);
-            T0 = fmaf(fu.y, odd ? S3[2] : r0, fu.x * (odd ? r0 : S3[0]));
-            T1 = fmaf(fu.y, odd ? S3[3] : r1, fu.x * (odd ? r1 : S3[1]));
-        }
-        // level 5: lanes s, s^2; bit1 = 0 keeps the first of the pair
-        const bool hi1 = (s >> 1) & 1;
-        const float r2 = __shfl_xor_sync(full, hi1 ? T0 : T1, 2);
-        float U;
-        {
-            const float2 fu = *(const float2*)(lut + 128 + o5);
-            U = fmaf(fu.y, hi1 ? T1 : r2, fu.x * (hi1 ? r2 : T0));
-        }
-        // root: lanes s, s^4 (both end with the same value)
-        const bool right = (s >> 2) & 1;
-        const float r3 = __shfl_xor_sync(full, U, 4);
-        float S;
-        {
-            const float2 fu = *(const float2*)(lut + 128 + o6);
-            S = fmaf(fu.y, right ? U : r3, fu.x * (right ? r3 : U));
-        }
-        const float rr = __half2float(((const __half*)pg)[t]);
-        if (s < 4) pbuf[t * kG + head] = t < valid ? rr * S * kLogitScale : -INFINITY;
+        // sum over the token's 8 subtrees; lanes s, s^1 end with head 2 b2 + b1
+        const float x0 = (b2 ? acc[2] : acc[0]) + __shfl_xor_sync(full, b2 ? acc[0] : acc[2], 4);
+        const float x1 = (b2 ? acc[3] : acc[1]) + __shfl_xor_sync(full, b2 ? acc[1] : acc[3], 4);
+        float y = (b1 ? x1 : x0) + __shfl_xor_sync(full, b1 ? x0 : x1, 2);
+        y += __shfl_xor_sync(full, y, 1);
+        if (!(s & 1)) pbuf[t * kG + 2 * b2 + b1] = t < valid ? y : -INFINITY;
     }
 }
 
@@ -541,27 +540,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const unsigned full = 0xffffffffu;
 
-    // cos/sin tables, one 256-byte row per code: leaf grid c*2pi/2^b_leaf in
-    // bytes 0..127, upper grid c*(pi/2)/(2^b_up-1) in bytes 128..255, each
-    // entry replicated for the 16 lanes of a half warp
-    {
-        constexpr int kRows = 256 + 64 + 16;
-        for (int e = tid; e < 2 * kRows; e += kThreads) {
-            const int row = e >> 1, upper = e & 1;
-            int tier_base, code, nleaf, nup;
-            if (row < 256) { tier_base = kLutT1; code = row; nleaf = 256; nup = 256; }
-            else if (row < 320) { tier_base = kLutT2; code = row - 256; nleaf = 16; nup = 64; }
-            else { tier_base = kLutT3; code = row - 320; nleaf = 8; nup = 16; }
-            double a = 0.0;   // angle / pi
-            if (!upper && code < nleaf) a = 2.0 * code / nleaf;
-            if (upper && code < nup) a = 0.5 * code / (nup - 1);
-            double sn, cs;
-            sincospi(a, &sn, &cs);
-            const float2 v = make_float2((float)cs, (float)sn);
-            float2* dst = (float2*)(smem + tier_base + code * kLutRow + upper * 128);
-#pragma unroll
-            for (int r = 0; r < 16; ++r) dst[r] = v;
+    // cos/sin tables: leaf grid c*2pi/2^b_leaf, upper grid c*(pi/2)/(2^b_up-1)
+    for (int e = tid; e < 2 * 256 + 64 + 16 + 16; e += kThreads) {
+        double a;   // angle / pi
+        int off, reps = 16;
+        if (e < 512) {   // T1 row e/2: leaf half, upper half
+            const int code = e >> 1, upper = e & 1;
+            a = upper ? 0.5 * code / 255 : 2.0 * code / 256;
+            off = kLutT1 + code * 256 + upper * 128;
+        } else if (e < 576) {
+            a = 0.5 * (e - 512) / 63;
+            off = kLutT2 + (e - 512) * 128;
+        } else if (e < 592) {
+            a = 0.5 * (e - 576) / 15;
+            off = kLutT3 + (e - 576) * 128;
+        } else {
+            a = 2.0 * (e - 592) / 16;
+            off = kLeafT2 + (e - 592) * 8;
+            reps = 1;
         }
+        double sn, cs;
+        sincospi(a, &sn, &cs);
+        const float2 v = make_float2((float)cs, (float)sn);
+        for (int r = 0; r < reps; ++r) ((float2*)(smem + off))[r] = v;
     }
     uint8_t* stage = smem + kStageOff + w * kStages * kStageBytes;
     float* pbuf = (float*)(smem + kPbufOff) + w * kPbufFloats;
@@ -592,12 +593,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
         const int len = p.seq_lens[b];
         const int32_t* ptab = p.page_table + (int64_t)g * p.total_pages + first;
 
-        // query-folded T2/T3 leaf tables for this unit (the previous segment
-        // ended with a barrier, so no warp still reads the old ones)
-        for (int e = tid; e < (16 + 8) * kLeaves; e += kThreads) {
-            const bool t3 = e >= 16 * kLeaves;
-            const int code = t3 ? (e - 16 * kLeaves) >> 6 : e >> 6, j = e & 63;
-            const float2 cs = *(const float2*)(smem + (t3 ? kLutT3 : kLutT2) + code * kLutRow);
+        // query-folded leaf table for this unit (the previous segment ended
+        // with a barrier, so no warp still reads the old one)
+        for (int e = tid; e < 16 * kLeaves; e += kThreads) {
+            const int code = e >> 6, j = e & 63;
+            const float2 cs = *(const float2*)(smem + kLeafT2 + code * 8);
             float v[kG];
 #pragma unroll
             for (int h = 0; h < kG; ++h) {
@@ -605,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
                 v[h] = fmaf(qh[2 * j + 1], cs.y, qh[2 * j] * cs.x);
             }
             const uint32_t off = ((uint32_t)code << 10) + 128u * (j >> 3) + 16u * ((j & 7) ^ (j >> 3));
-            *(float4*)(smem + kFoldOff + (t3 ? kFoldT3 : kFoldT2) + off) = make_float4(v[0], v[1], v[2], v[3]);
+            *(float4*)(smem + kFoldOff + off) = make_float4(v[0], v[1], v[2], v[3]);
         }
         for (int e = tid; e < 2 * kLeaves; e += kThreads) {   // q for T1 leaves
             const int odd = e >= kLeaves, j = e & 63, sj = j >> 3, ij = j & 7;
