@@ -73,7 +73,7 @@ constexpr int kPbufFloats = 16 * kG + 2 * kG;   // p*scale per (token, head); al
 constexpr int kFoldOff = (kPbufOff + kWarps * kPbufFloats * 4 + 127) / 128 * 128;
 constexpr int kFoldBytes = 16 * 1024;
 // The unit's query for T1 leaves: even dims and odd dims of leaf j = 8s + i in
-// two arrays of 16-byte entries (4 heads) at entry 8s + ((i + s) & 7), so the 8
+// two 1 KB arrays of 16-byte entries (4 heads) at byte 144 s ^ 16 i, so the 8
 // subtree lanes of a token read 8 distinct banks.
 constexpr int kQOff = kFoldOff + kFoldBytes;
 constexpr int kQBytes = 2 * kLeaves * 16;
@@ -250,12 +250,11 @@ struct WarpState {
 // Offsets of the 8 leaf and 8 upper codes of one subtree block.  T1: byte
 // offset code << 8 | replica << 3 into its 256-byte rows; T2/T3 upper codes:
 // code << 7 | replica << 3; base_rep = (lane & 15) << 3.  T2/T3 leaves: offset
-// (T3 code c read as T2 code 2c) into the
-// query-folded table, (code << 10 | 144 s) ^ 16 i for leaf i of subtree s,
-// with fold_lane = 144 s.
+// (T3 code c read as T2 code 2c) into the query-folded table,
+// code << 10 | fl[i] for leaf i of subtree s, fl[i] = 144 s ^ 16 i.
 template <int T>
-__device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uint32_t base_rep, uint32_t fold_lane,
-                                              uint32_t (&lo)[8], uint32_t (&uo)[8])
+__device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uint32_t base_rep,
+                                              const uint32_t (&fl)[8], uint32_t (&lo)[8], uint32_t (&uo)[8])
 {
     if (T == 1) {   // byte codes: one permute places the code in bits 8..15
         const uint4 w = *(const uint4*)(codes + blk * 16);
@@ -271,7 +270,7 @@ __device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uin
         const uint32_t h = *(const uint16_t*)(codes + kP * 64 + blk * 2);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            lo[j] = ((((w.x >> (4 * j)) & 15u) << 10) | fold_lane) ^ (16u * j);
+            lo[j] = (((w.x >> (4 * j)) & 15u) << 10) | fl[j];
             uo[j] = (((w.y >> (4 * j)) & 15u) << 7) | (((h >> (2 * j)) & 3u) << 11) | base_rep;
         }
     } else {
@@ -280,7 +279,7 @@ __device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uin
         const uint32_t l1 = codes[kP * 48 + blk];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            lo[j] = ((((l2 >> (2 * j)) & 3u) << 11) | (((l1 >> j) & 1u) << 13) | fold_lane) ^ (16u * j);
+            lo[j] = (((l2 >> (2 * j)) & 3u) << 11) | (((l1 >> j) & 1u) << 13) | fl[j];
             uo[j] = (((u >> (4 * j)) & 15u) << 7) | base_rep;
         }
     }
@@ -311,7 +310,7 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 }
 
 // Logits of the 16 tokens of one page of tier T staged at `pg`, written in the
-// log2 domain to pbuf[t * kG + head] (-inf for slots past `valid`).  Lane
+// log2 domain to pbuf[t * kG + head].  Lane
 // (k, s) handles subtree s of tokens 4 pass + k for all 4 heads, top down:
 // the tree's value r S_root is the sum over leaves of (product of the factors
 // on the leaf's path: cos(psi) into a left child, sin(psi) into a right one)
@@ -320,7 +319,8 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 // multiply-add per leaf (T2/T3, whose leaf terms are read from the
 // query-folded tables) or per dimension (T1).
 template <int T>
-__device__ __forceinline__ void page_logits(const uint8_t* pg, int valid, const uint8_t* smem, float* pbuf, int lane)
+__device__ __forceinline__ void page_logits(const uint8_t* pg, const uint8_t* smem, float* pbuf, int lane,
+                                            const uint32_t (&fl)[8])
 {
     const unsigned full = 0xffffffffu;
     const int k = lane >> 3, s = lane & 7;
@@ -330,9 +330,6 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, int valid, const 
     const uint8_t* lut = smem + kBase;
     const uint8_t* lut_up = lut + kUp;
     const uint32_t rep = (uint32_t)(lane & 15) << 3;
-    const uint32_t fold_lane = 144u * (uint32_t)s;
-    const float4* qe = (const float4*)(smem + kQOff);   // q[2j] of the 4 heads
-    const float4* qo = qe + kLeaves;                     // q[2j + 1]
     const uint8_t* codes = pg + Tier<1>::f.off_codes;
     // ancestors of subtree s: level-4 node s>>1, level-5 node s>>2, the root;
     // the subtree lies on their right (sin, byte 4 of the entry) or left side
@@ -343,7 +340,7 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, int valid, const 
     for (int pass = 0; pass < 4; ++pass) {
         const int t = pass * 4 + k;
         uint32_t lo[8], uo[8];
-        block_offsets<T>(codes, t * 8 + s, rep, fold_lane, lo, uo);
+        block_offsets<T>(codes, t * 8 + s, rep, fl, lo, uo);
         // top codes: block i carries top node i (level 4 nodes 0..3, level 5
         // nodes 0..1, root)
         const uint32_t o4 = __shfl_sync(full, uo[7], (lane & ~7) | (s >> 1));
@@ -378,8 +375,8 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, int valid, const 
             if (T == 1) {
                 const float2 f = *(const float2*)(lut + lo[j]);
                 const float kx = wl[j] * f.x, ky = wl[j] * f.y;
-                const int e = 8 * s + ((j + s) & 7);
-                const float4 ev = qe[e], od = qo[e];
+                const float4 ev = *(const float4*)(smem + kQOff + fl[j]);          // q[2j], 4 heads
+                const float4 od = *(const float4*)(smem + kQOff + 1024 + fl[j]);   // q[2j + 1]
                 const float qev[kG] = {ev.x, ev.y, ev.z, ev.w}, qod[kG] = {od.x, od.y, od.z, od.w};
 #pragma unroll
                 for (int h = 0; h < kG; ++h) acc[h] = fmaf(qod[h], ky, j == 0 ? qev[h] * kx : fmaf(qev[h], kx, acc[h]));
@@ -395,7 +392,7 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, int valid, const 
         const float x1 = (b2 ? acc[3] : acc[1]) + __shfl_xor_sync(full, b2 ? acc[1] : acc[3], 4);
         float y = (b1 ? x1 : x0) + __shfl_xor_sync(full, b1 ? x0 : x1, 2);
         y += __shfl_xor_sync(full, y, 1);
-        if (!(s & 1)) pbuf[t * kG + 2 * b2 + b1] = t < valid ? y : -INFINITY;
+        if (!(s & 1)) pbuf[t * kG + 2 * b2 + b1] = y;
     }
 }
 
@@ -403,18 +400,22 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, int valid, const 
 // are tier-specialised; the softmax and the value MMAs are one copy of code
 // for all tiers apart from the value conversion.
 __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int valid, const uint8_t* smem, float* pbuf,
-                                             int lane, WarpState& st)
+                                             int lane, const uint32_t (&fl)[8], WarpState& st)
 {
     const unsigned full = 0xffffffffu;
     const int k = lane >> 3, s = lane & 7;
     const int head = (s & 1) * 2 + ((s >> 1) & 1);
-    if (tier == 1) page_logits<1>(pg, valid, smem, pbuf, lane);
-    else if (tier == 2) page_logits<2>(pg, valid, smem, pbuf, lane);
-    else page_logits<3>(pg, valid, smem, pbuf, lane);
+    // `valid` waits in the buffer's spare word while the logits hold the registers
+    if (lane == 0) ((int*)pbuf)[16 * kG + kG] = valid;
+    if (tier == 1) page_logits<1>(pg, smem, pbuf, lane, fl);
+    else if (tier == 2) page_logits<2>(pg, smem, pbuf, lane, fl);
+    else page_logits<3>(pg, smem, pbuf, lane, fl);
     __syncwarp();
+    valid = ((const int*)pbuf)[16 * kG + kG];
     float lg[4];
 #pragma unroll
-    for (int pass = 0; pass < 4; ++pass) lg[pass] = pbuf[(pass * 4 + k) * kG + head];
+    for (int pass = 0; pass < 4; ++pass)   // slots past `valid` (last page) get -inf
+        lg[pass] = pass * 4 + k < valid ? pbuf[(pass * 4 + k) * kG + head] : -INFINITY;
     __syncwarp();
     // online softmax for this lane's head (lanes k = 0..3 share it)
     float pm = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
@@ -499,6 +500,7 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
     } else {   // T2 and T3 share the int4 row format
         const uint8_t* vrow = pg + (tier == 2 ? Tier<2>::f.off_v : Tier<3>::f.off_v);
         const __half2 bias = __floats2half2_rn(-1032.f, -1032.f);
+        const __half2 inv16 = __floats2half2_rn(0.0625f, 0.0625f), bias16 = __floats2half2_rn(-72.f, -72.f);
         // tokens 2i, 2i+1 share a 128-byte block; chunk g ^ (2i & 6) holds 8
         // bytes of each.  Pairs c and c + 4 both give 2i & 6 = 2c.
         const int ch = 16 * (g ^ (2 * c));
@@ -516,15 +518,19 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
             const uint32_t sel = (uint32_t)(b | ((4 + b) << 8));
             const uint32_t xy = __byte_perm(xs[wi], ys[wi], sel);
             const uint32_t zw = __byte_perm(zs[wi], ws[wi], sel);
+            // low nibble: f16 1024 + u; high nibble in place: f16 1024 + 16 u,
+            // scaled by 1/16 in the bias step (all exact in f16)
             uint32_t a[4];
             a[0] = (xy & 0x000F000Fu) | 0x64006400u;
-            a[1] = ((xy >> 4) & 0x000F000Fu) | 0x64006400u;
+            a[1] = (xy & 0x00F000F0u) | 0x64006400u;
             a[2] = (zw & 0x000F000Fu) | 0x64006400u;
-            a[3] = ((zw >> 4) & 0x000F000Fu) | 0x64006400u;
+            a[3] = (zw & 0x00F000F0u) | 0x64006400u;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                __half2 hv = __hadd2(*(const __half2*)&a[i], bias);
-                a[i] = *(const uint32_t*)&hv;
+            for (int i = 0; i < 4; i += 2) {
+                const __half2 lo = __hadd2(*(const __half2*)&a[i], bias);
+                const __half2 hi = __hfma2(*(const __half2*)&a[i + 1], inv16, bias16);
+                a[i] = *(const uint32_t*)&lo;
+                a[i + 1] = *(const uint32_t*)&hi;
             }
             mma_16816(st.acc[m], a, bh0, bh1);
             mma_16816(st.acc[m], a, bl0, bl1);
@@ -564,6 +570,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
         const float2 v = make_float2((float)cs, (float)sn);
         for (int r = 0; r < reps; ++r) ((float2*)(smem + off))[r] = v;
     }
+    // per-lane offsets of leaf i of subtree s = lane & 7 in the folded table
+    // and the T1 query arrays
+    uint32_t fl[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) fl[i] = (144u * (uint32_t)(lane & 7)) ^ (16u * i);
     uint8_t* stage = smem + kStageOff + w * kStages * kStageBytes;
     float* pbuf = (float*)(smem + kPbufOff) + w * kPbufFloats;
     const uint32_t bar0 = smem_u32(smem + kBarOff + w * kStages * 8);
@@ -612,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
             float v[kG];
 #pragma unroll
             for (int h = 0; h < kG; ++h) v[h] = p.q[((int64_t)b * p.H_q + g * kG + h) * kD + 2 * j + odd];
-            ((float4*)(smem + kQOff))[odd * kLeaves + 8 * sj + ((ij + sj) & 7)] = make_float4(v[0], v[1], v[2], v[3]);
+            *(float4*)(smem + kQOff + 1024 * odd + ((144 * sj) ^ (16 * ij))) = make_float4(v[0], v[1], v[2], v[3]);
         }
         __syncthreads();
         WarpState st;
@@ -687,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
             const uint8_t* pg = stage + cur * kStageBytes;
             const int valid = min(kP, len - lp_cur * kP);
             const int t = entry_tier(e_cur);
-            process_page(pg, t, valid, smem, pbuf, lane, st);
+            process_page(pg, t, valid, smem, pbuf, lane, fl, st);
             cur ^= 1;
             lp_cur = lp_nxt;
             e_cur = e_nxt;
