@@ -78,7 +78,8 @@ constexpr int kFoldBytes = 16 * 1024;
 constexpr int kQOff = kFoldOff + kFoldBytes;
 constexpr int kQBytes = 2 * kLeaves * 16;
 constexpr int kBarOff = kQOff + kQBytes;
-constexpr int kSmemBytes = kBarOff + kWarps * kStages * 8;
+constexpr int kSliceOff = kBarOff + kWarps * kStages * 8;   // per-warp slice weights
+constexpr int kSmemBytes = kSliceOff + kWarps * 4;
 static_assert(kStageOff % 128 == 0 && kPbufOff % 16 == 0 && kFoldOff % 128 == 0 && kQOff % 128 == 0 &&
                   kBarOff % 8 == 0,
               "smem alignment");
@@ -238,6 +239,15 @@ __device__ inline int find_unit(const int32_t* us, int n_units, int32_t x)
 __device__ inline int32_t cta_bound(int c, int32_t P, int n_cta)
 {
     return (int32_t)(((int64_t)c * P) / n_cta);
+}
+
+// Work of a page by tier, for splitting a CTA's pages among its warps: a T1
+// page takes about 4/3 of the time of a T2 or T3 page; dropped pages are
+// skipped.
+__device__ __forceinline__ uint32_t page_weight(int32_t e)
+{
+    const int t = entry_tier(e);
+    return t == 0 ? 0u : t == 1 ? 4u : 3u;
 }
 
 // ------------------------------------------------------------- page work --
@@ -604,6 +614,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
         const int len = p.seq_lens[b];
         const int32_t* ptab = p.page_table + (int64_t)g * p.total_pages + first;
 
+        // Split [pa, pe) among the warps by weight.  Warp w first sums slice w
+        // (pages pa + n k / 16 for k = w, w + 1); after the barrier each warp
+        // finds where the running weight crosses W w / 16 and W (w + 1) / 16.
+        // The split depends only on the page table, so results are
+        // reproducible bit for bit.
+        uint32_t* wsum = (uint32_t*)(smem + kSliceOff);
+        const int32_t n_seg = pe - pa;
+        auto slice_start = [&](int k) -> int32_t { return pa + (int32_t)(((int64_t)n_seg * k) / kWarps); };
+        {
+            uint32_t sum = 0;
+            for (int32_t i = slice_start(w) + lane; i < slice_start(w + 1); i += 32) sum += page_weight(ptab[i]);
+            sum = __reduce_add_sync(full, sum);
+            if (lane == 0) wsum[w] = sum;
+        }
         // query-folded leaf table for this unit (the previous segment ended
         // with a barrier, so no warp still reads the old one)
         for (int e = tid; e < 16 * kLeaves; e += kThreads) {
@@ -626,6 +650,44 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
             *(float4*)(smem + kQOff + 1024 * odd + ((144 * sj) ^ (16 * ij))) = make_float4(v[0], v[1], v[2], v[3]);
         }
         __syncthreads();
+        int32_t ra, rb;   // this warp's unit-local page range
+        {
+            const int64_t sl = lane < kWarps ? (int64_t)wsum[lane] : 0;
+            int64_t incl = sl;   // inclusive prefix over the slices
+#pragma unroll
+            for (int o = 1; o < kWarps; o <<= 1) {
+                const int64_t y = __shfl_up_sync(full, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int64_t W = __shfl_sync(full, incl, kWarps - 1);
+            // first page whose running weight (itself included) exceeds W k / 16
+            auto boundary = [&](int k) -> int32_t {
+                if (k == 0) return pa;
+                if (k == kWarps) return pe;
+                const int64_t T = W * k / kWarps;
+                const uint32_t over = __ballot_sync(full, lane < kWarps && incl > T);
+                if (over == 0) return pe;
+                const int j = __ffs(over) - 1;
+                int64_t run = __shfl_sync(full, incl, j) - __shfl_sync(full, sl, j);
+                const int32_t i1 = slice_start(j + 1);
+                for (int32_t base = slice_start(j); base < i1; base += 32) {
+                    const int32_t i = base + lane;
+                    uint32_t c = i < i1 ? page_weight(ptab[i]) : 0u;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const uint32_t y = __shfl_up_sync(full, c, o);
+                        if (lane >= o) c += y;
+                    }
+                    const uint32_t le = __ballot_sync(full, i < i1 && run + (int64_t)c <= T);
+                    const int n_le = __popc(le), n_in = min(32, i1 - base);
+                    if (n_le < n_in) return base + n_le;
+                    run += __shfl_sync(full, c, 31);
+                }
+                return i1;
+            };
+            ra = boundary(w);
+            rb = boundary(w + 1);
+        }
         WarpState st;
         st.m = -INFINITY;
         st.l = 0.f;
@@ -634,15 +696,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
 #pragma unroll
             for (int i = 0; i < 4; ++i) st.acc[m][i] = 0.f;
 
-        // this warp's pages: pa + w + kWarps*i.  Entries are read 32 at a time.
+        // this warp's pages: [ra, rb).  Entries are read 32 at a time.
         struct Cursor {
             int ebase;
             int32_t ent;
             uint32_t mask;
         };
         auto refill = [&](Cursor& cu) {
-            const int32_t lp = pa + w + kWarps * (cu.ebase + lane);
-            cu.ent = lp < pe ? ptab[lp] : 0;
+            const int32_t lp = ra + cu.ebase + lane;
+            cu.ent = lp < rb ? ptab[lp] : 0;
             const int t = entry_tier(cu.ent);
             bool ok = t != 0;
             if (ok && entry_page(cu.ent) >= p.pool_pages[t]) {
@@ -654,12 +716,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
         auto advance = [&](Cursor& cu, int32_t& lp, int32_t& e) -> bool {
             while (cu.mask == 0) {
                 cu.ebase += 32;
-                if (pa + w + kWarps * cu.ebase >= pe) return false;
+                if (ra + cu.ebase >= rb) return false;
                 refill(cu);
             }
             const int j = __ffs(cu.mask) - 1;
             cu.mask &= cu.mask - 1;
-            lp = pa + w + kWarps * (cu.ebase + j);
+            lp = ra + cu.ebase + j;
             e = __shfl_sync(full, cu.ent, j);
             return true;
         };
