@@ -275,21 +275,26 @@ __device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uin
             uo[j] = __byte_perm(w.z, base_rep, 0x7604 | (j << 4));
             uo[4 + j] = __byte_perm(w.w, base_rep, 0x7604 | (j << 4));
         }
-    } else if (T == 2) {
+    } else if (T == 2) {   // upper code j = bits 6j..6j+5 of the 48-bit field h:w.y
         const uint2 w = *(const uint2*)(codes + blk * 8);
         const uint32_t h = *(const uint16_t*)(codes + kP * 64 + blk * 2);
+        constexpr uint32_t kUpMask = 63u << 7;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            lo[j] = (((w.x >> (4 * j)) & 15u) << 10) | fl[j];
-            uo[j] = (((w.y >> (4 * j)) & 15u) << 7) | (((h >> (2 * j)) & 3u) << 11) | base_rep;
-        }
-    } else {
+        for (int j = 0; j < 8; ++j) lo[j] = (((w.x >> (4 * j)) & 15u) << 10) | fl[j];
+        uo[0] = ((w.y << 7) & kUpMask) | base_rep;
+        uo[1] = ((w.y << 1) & kUpMask) | base_rep;
+        uo[2] = ((w.y >> 5) & kUpMask) | base_rep;
+        uo[3] = ((w.y >> 11) & kUpMask) | base_rep;
+        uo[4] = ((w.y >> 17) & kUpMask) | base_rep;
+        uo[5] = (__funnelshift_r(w.y, h, 23) & kUpMask) | base_rep;
+        uo[6] = ((h << 3) & kUpMask) | base_rep;
+        uo[7] = ((h >> 3) & kUpMask) | base_rep;
+    } else {   // leaf code j = bits 3j..3j+2 of the 24-bit field l8:l16
         const uint32_t u = *(const uint32_t*)(codes + blk * 4);
-        const uint32_t l2 = *(const uint16_t*)(codes + kP * 32 + blk * 2);
-        const uint32_t l1 = codes[kP * 48 + blk];
+        const uint32_t lf = *(const uint16_t*)(codes + kP * 32 + blk * 2) | ((uint32_t)codes[kP * 48 + blk] << 16);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            lo[j] = (((l2 >> (2 * j)) & 3u) << 11) | (((l1 >> j) & 1u) << 13) | fl[j];
+            lo[j] = (((lf >> (3 * j)) & 7u) << 11) | fl[j];
             uo[j] = (((u >> (4 * j)) & 15u) << 7) | base_rep;
         }
     }

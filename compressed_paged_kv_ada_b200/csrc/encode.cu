@@ -139,40 +139,38 @@ __device__ void encode_token(const EncParams& p, int64_t i, int g, uint8_t* page
             word |= code << (8 * b);
         }
         ((uint32_t*)codes)[slot * 32 + lane] = word;
-    } else if (T == 2) {   // u32 leaf nibbles, u32 upper low nibbles | u16 upper high bits
-        if (lane < 16) {
-            const int s = lane >> 1, w = lane & 1;
-            uint32_t word = 0;
+    } else if (T == 2) {   // u32 leaf nibbles, low 32 bits of the 48-bit upper field | u16 its high bits
+        if (lane < 24) {
+            const int s = lane < 16 ? lane >> 1 : lane - 16;
+            uint64_t uf = 0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                word |= (w == 0 ? (uint32_t)sleaf[8 * s + j] : (block_up(sup, s, j) & 15u)) << (4 * j);
-            ((uint32_t*)codes)[slot * 16 + lane] = word;
-        } else if (lane < 24) {
-            const int s = lane - 16;
-            uint32_t h = 0;
+            for (int j = 0; j < 8; ++j) uf |= (uint64_t)block_up(sup, s, j) << (6 * j);
+            if (lane < 16) {
+                uint32_t word = (uint32_t)uf;
+                if ((lane & 1) == 0) {
+                    word = 0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) h |= (block_up(sup, s, j) >> 4) << (2 * j);
-            ((uint16_t*)(codes + kP * 64))[slot * 8 + s] = (uint16_t)h;
+                    for (int j = 0; j < 8; ++j) word |= (uint32_t)sleaf[8 * s + j] << (4 * j);
+                }
+                ((uint32_t*)codes)[slot * 16 + lane] = word;
+            } else {
+                ((uint16_t*)(codes + kP * 64))[slot * 8 + s] = (uint16_t)(uf >> 32);
+            }
         }
-    } else {   // u32 upper nibbles | u16 leaf low 2 bits | u8 leaf high bit
+    } else {   // u32 upper nibbles | u16 low and u8 high bits of the 24-bit leaf field
         if (lane < 8) {
             const int s = lane;
             uint32_t word = 0;
 #pragma unroll
             for (int j = 0; j < 8; ++j) word |= block_up(sup, s, j) << (4 * j);
             ((uint32_t*)codes)[slot * 8 + s] = word;
-        } else if (lane < 16) {
-            const int s = lane - 8;
-            uint32_t lo = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) lo |= ((uint32_t)sleaf[8 * s + j] & 3u) << (2 * j);
-            ((uint16_t*)(codes + kP * 32))[slot * 8 + s] = (uint16_t)lo;
         } else if (lane < 24) {
-            const int s = lane - 16;
-            uint32_t hi = 0;
+            const int s = lane < 16 ? lane - 8 : lane - 16;
+            uint32_t lf = 0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) hi |= ((uint32_t)sleaf[8 * s + j] >> 2) << j;
-            (codes + kP * 48)[slot * 8 + s] = (uint8_t)hi;
+            for (int j = 0; j < 8; ++j) lf |= (uint32_t)sleaf[8 * s + j] << (3 * j);
+            if (lane < 16) ((uint16_t*)(codes + kP * 32))[slot * 8 + s] = (uint16_t)lf;
+            else (codes + kP * 48)[slot * 8 + s] = (uint8_t)(lf >> 16);
         }
     }
     // value row: position p holds channel v_channel_at(p); 16-byte chunks are

@@ -50,10 +50,11 @@
  *  nodes, the root), U[7][7] = 0.  Code planes, each [16 tokens][8 blocks]
  *  [width], little-endian:
  *    T1: width 16: bytes 0..7 = L[s][0..7], bytes 8..15 = U[s][0..7];
- *    T2: width 8: u32 nibble j = L[s][j], u32 nibble j = U[s][j] & 15;
- *        width 2: u16 bits 2j..2j+1 = U[s][j] >> 4;
- *    T3: width 4: u32 nibble j = U[s][j]; width 2: u16 bits 2j..2j+1 =
- *        L[s][j] & 3; width 1: u8 bit j = L[s][j] >> 2.
+ *    T2: width 8: u32 nibble j = L[s][j], then the low 32 bits of the
+ *        48-bit field F with bits 6j..6j+5 = U[s][j]; width 2: u16 = F >> 32;
+ *    T3: width 4: u32 nibble j = U[s][j]; width 2: u16 = G & 0xFFFF and
+ *        width 1: u8 = G >> 16 of the 24-bit field G with bits 3j..3j+2 =
+ *        L[s][j].
  *  Value row position p = 16g + 2m + h (g, m = 0..7, h = 0..1) holds channel
  *  16m + g + 8h.  int8 (T1): token r has a 128-byte row whose 16-byte chunk g
  *  (positions 16g..16g+15) is stored at chunk g ^ (r & 6).  int4 (T2, T3):

@@ -389,10 +389,12 @@ static uint64_t get_le(const uint8_t* src, int nbytes)
 /* Store one token (d = 128) into slot `slot` of a page of tier t (1..3).
  * Code planes (each [16 tokens][8 blocks][width] bytes, in this order):
  *   T1: width 16: bytes 0..7 = L[s][0..7], bytes 8..15 = U[s][0..7];
- *   T2: width 8: u32 with nibble j = L[s][j], then u32 with nibble j =
- *       U[s][j] & 15;  width 2: u16 with bits 2j..2j+1 = U[s][j] >> 4;
- *   T3: width 4: u32 with nibble j = U[s][j];  width 2: u16 with bits
- *       2j..2j+1 = L[s][j] & 3;  width 1: u8 with bit j = L[s][j] >> 2.
+ *   T2: width 8: u32 with nibble j = L[s][j], then the low 32 bits of the
+ *       48-bit field with bits 6j..6j+5 = U[s][j];  width 2: u16 = the high
+ *       16 bits of that field;
+ *   T3: width 4: u32 with nibble j = U[s][j];  width 2: u16 = the low 16 bits
+ *       of the 24-bit field with bits 3j..3j+2 = L[s][j];  width 1: u8 = its
+ *       high 8 bits.
  * Multi-byte fields are little-endian.  Value row position p holds channel
  * v_channel_at(p), stored at v_byte_at (int4: two's complement nibbles). */
 void orc_pack_token(int t, int slot, const uint8_t* leaf, const uint8_t* up, uint16_t r16,
@@ -411,24 +413,22 @@ void orc_pack_token(int t, int slot, const uint8_t* leaf, const uint8_t* up, uin
                 c[blk * 16 + 8 + j] = U[s][j];
             }
         } else if (t == 2) {
-            uint64_t a = 0, b = 0;
+            uint64_t lf = 0, uf = 0;
             for (int j = 0; j < 8; ++j) {
-                a |= (uint64_t)L[s][j] << (4 * j);
-                a |= (uint64_t)(U[s][j] & 15) << (32 + 4 * j);
-                b |= (uint64_t)(U[s][j] >> 4) << (2 * j);
+                lf |= (uint64_t)L[s][j] << (4 * j);
+                uf |= (uint64_t)U[s][j] << (6 * j);
             }
-            put_le(c + blk * 8, 8, a);
-            put_le(c + ORC_PAGE * 8 * 8 + blk * 2, 2, b);
+            put_le(c + blk * 8, 8, lf | (uf << 32));
+            put_le(c + ORC_PAGE * 8 * 8 + blk * 2, 2, uf >> 32);
         } else {
-            uint64_t a = 0, b = 0, e = 0;
+            uint64_t uf = 0, lf = 0;
             for (int j = 0; j < 8; ++j) {
-                a |= (uint64_t)U[s][j] << (4 * j);
-                b |= (uint64_t)(L[s][j] & 3) << (2 * j);
-                e |= (uint64_t)(L[s][j] >> 2) << j;
+                uf |= (uint64_t)U[s][j] << (4 * j);
+                lf |= (uint64_t)L[s][j] << (3 * j);
             }
-            put_le(c + blk * 4, 4, a);
-            put_le(c + ORC_PAGE * 8 * 4 + blk * 2, 2, b);
-            put_le(c + ORC_PAGE * 8 * 6 + blk, 1, e);
+            put_le(c + blk * 4, 4, uf);
+            put_le(c + ORC_PAGE * 8 * 4 + blk * 2, 2, lf & 0xffff);
+            put_le(c + ORC_PAGE * 8 * 6 + blk, 1, lf >> 16);
         }
     }
     for (int p = 0; p < ORC_D; ++p) {
@@ -456,16 +456,18 @@ void orc_unpack_token(int t, int slot, const uint8_t* page, uint8_t* leaf, uint8
             }
         } else if (t == 2) {
             uint64_t a = get_le(c + blk * 8, 8), b = get_le(c + ORC_PAGE * 8 * 8 + blk * 2, 2);
+            uint64_t uf = (a >> 32) | (b << 32);
             for (int j = 0; j < 8; ++j) {
                 L[s][j] = (uint8_t)((a >> (4 * j)) & 15);
-                U[s][j] = (uint8_t)(((a >> (32 + 4 * j)) & 15) | (((b >> (2 * j)) & 3) << 4));
+                U[s][j] = (uint8_t)((uf >> (6 * j)) & 63);
             }
         } else {
             uint64_t a = get_le(c + blk * 4, 4), b = get_le(c + ORC_PAGE * 8 * 4 + blk * 2, 2),
                      e = get_le(c + ORC_PAGE * 8 * 6 + blk, 1);
+            uint64_t lf = b | (e << 16);
             for (int j = 0; j < 8; ++j) {
                 U[s][j] = (uint8_t)((a >> (4 * j)) & 15);
-                L[s][j] = (uint8_t)(((b >> (2 * j)) & 3) | (((e >> j) & 1) << 2));
+                L[s][j] = (uint8_t)((lf >> (3 * j)) & 7);
             }
         }
     }

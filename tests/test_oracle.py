@@ -401,12 +401,14 @@ def test_pack_unpack_roundtrip_and_independent_layout():
                     assert page[64 + 16 * blk:64 + 16 * blk + 16].tolist() == L[s] + U[s]
                 elif t == 2:
                     assert rd(64 + 8 * blk, 4) == sum(L[s][j] << (4 * j) for j in range(8))
-                    assert rd(68 + 8 * blk, 4) == sum((U[s][j] & 15) << (4 * j) for j in range(8))
-                    assert rd(64 + 1024 + 2 * blk, 2) == sum((U[s][j] >> 4) << (2 * j) for j in range(8))
+                    uf = sum(U[s][j] << (6 * j) for j in range(8))
+                    assert rd(68 + 8 * blk, 4) == uf & 0xFFFFFFFF
+                    assert rd(64 + 1024 + 2 * blk, 2) == uf >> 32
                 else:
                     assert rd(64 + 4 * blk, 4) == sum(U[s][j] << (4 * j) for j in range(8))
-                    assert rd(64 + 512 + 2 * blk, 2) == sum((L[s][j] & 3) << (2 * j) for j in range(8))
-                    assert rd(64 + 768 + blk, 1) == sum((L[s][j] >> 2) << j for j in range(8))
+                    lf = sum(L[s][j] << (3 * j) for j in range(8))
+                    assert rd(64 + 512 + 2 * blk, 2) == lf & 0xFFFF
+                    assert rd(64 + 768 + blk, 1) == lf >> 16
             voff = 64 + 16 * {1: 128, 2: 80, 3: 56}[t]
             for p in range(128):
                 ch = 16 * ((p >> 1) & 7) + (p >> 4) + 8 * (p & 1)
