@@ -90,9 +90,12 @@ static_assert((2 * kWarps * kG + kWarps * kG * kD) * 4 <= kWarps * kStages * kSt
 constexpr float kLn2 = 0.6931471805599453f;
 // log2(e) / sqrt(128): logits are kept in the log2 domain
 constexpr float kLogitScale = 0.12751743082459868f;
-// the value weights p * scale are multiplied by 2^12 before the f16 split
+// The value weights p * vscale are multiplied by a power of two sc before the
+// f16 hi/lo split: 2^12 to start with, lowered (with the accumulators
+// rescaled) when a page brings a scale with vscale * sc > 2^15, so that a
+// weight (p <= 1) never leaves the f16 range.
 constexpr float kPScale = 4096.0f;
-constexpr float kInvPScale = 1.0f / 4096.0f;
+constexpr float kWeightMax = 32768.0f;
 
 constexpr long kWaitLimit = 1L << 22;
 
@@ -254,8 +257,15 @@ __device__ __forceinline__ uint32_t page_weight(int32_t e)
 struct WarpState {
     float m;             // running max (log2 domain) of this lane's head
     float l;             // running sum of this lane's tokens
-    float acc[8][4];     // MMA accumulators: tile m = dims 16m..16m+15
+    float sc;            // power of two: value weights are p * vscale * sc
+    float acc[8][4];     // MMA accumulators (in units of 1 / sc): tile m = dims 16m..16m+15
 };
+
+// Largest power of two <= x (x positive and normal).
+__device__ __forceinline__ float pow2_floor(float x)
+{
+    return __int_as_float(__float_as_int(x) & 0x7f800000);
+}
 
 // Offsets of the 8 leaf and 8 upper codes of one subtree block.  T1: byte
 // offset code << 8 | replica << 3 into its 256-byte rows; T2/T3 upper codes:
@@ -439,24 +449,43 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
     const float m_new = fmaxf(st.m, pm);
     const float alpha = fast_exp2(st.m - m_new);   // st.m = -inf on the first page -> 0
     st.m = m_new;
-    float psum = 0.f;
     const __half* vs = (const __half*)(pg + 2 * kP);
+    float wv[4];   // vscale * sc of this lane's tokens
+    bool big = false;
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+        const int t = pass * 4 + k;   // slots past `valid` may hold stale scales: weight exactly 0
+        wv[pass] = t < valid ? __half2float(vs[t]) * st.sc : 0.f;
+        big |= wv[pass] > kWeightMax;
+    }
+    float alpha_acc = alpha;
+    if (__any_sync(full, big)) {   // rare: lower sc so every weight fits f16
+        float vm = fmaxf(fmaxf(wv[0], wv[1]), fmaxf(wv[2], wv[3]));
+        vm = fmaxf(vm, __shfl_xor_sync(full, vm, 8));
+        vm = fmaxf(vm, __shfl_xor_sync(full, vm, 16));
+        const float ratio = pow2_floor(kWeightMax / vm);   // exact: both powers of two scale exactly
+        st.sc *= ratio;
+        alpha_acc *= ratio;
+#pragma unroll
+        for (int pass = 0; pass < 4; ++pass) wv[pass] *= ratio;
+    }
+    float psum = 0.f;
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
         const float pv = fast_exp2(lg[pass] - m_new);
         psum += pv;
-        const int t = pass * 4 + k;   // slots past `valid` may hold stale scales: weight exactly 0
-        if (s < 4) pbuf[t * kG + head] = t < valid ? pv * __half2float(vs[t]) * kPScale : 0.f;
+        const int t = pass * 4 + k;
+        if (s < 4) pbuf[t * kG + head] = pv * wv[pass];
     }
     st.l = st.l * alpha + psum;
-    if (lane < 4) pbuf[16 * kG + head] = alpha;
+    if (lane < 4) pbuf[16 * kG + head] = alpha_acc;
     __syncwarp();
 
     // values on the tensor cores.  Thread (g, c): B columns = head g (g < 4),
     // rows = tokens 2c, 2c+1 (b0) and 2c+8, 2c+9 (b1); accumulator columns =
     // heads 2c, 2c+1.
     const int g = lane >> 2, c = lane & 3;
-    if (__any_sync(full, alpha != 1.f)) {   // a running max moved: rescale (rare after the first pages)
+    if (__any_sync(full, alpha_acc != 1.f)) {   // a running max or sc moved: rescale (rare after the first pages)
         const float2 al = *(const float2*)(pbuf + 16 * kG + 2 * (c & 1));
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
@@ -696,6 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
         WarpState st;
         st.m = -INFINITY;
         st.l = 0.f;
+        st.sc = kPScale;
 #pragma unroll
         for (int m = 0; m < 8; ++m)
 #pragma unroll
@@ -786,12 +816,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
             }
             // accumulator (tile m, i): dim 16m + g + 8*(i >> 1), head 2c + (i & 1)
             const int gq = lane >> 2, cq = lane & 3;
+            const float inv_sc = 1.0f / st.sc;   // exact: sc is a power of two
             if (cq < 2) {
 #pragma unroll
                 for (int m = 0; m < 8; ++m)
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        ms_o[(w * kG + 2 * cq + (i & 1)) * kD + 16 * m + gq + 8 * (i >> 1)] = st.acc[m][i];
+                        ms_o[(w * kG + 2 * cq + (i & 1)) * kD + 16 * m + gq + 8 * (i >> 1)] = st.acc[m][i] * inv_sc;
             }
         }
         __syncthreads();
@@ -813,7 +844,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
             }
             if (pa == 0 && seg_end == ue) {   // the whole unit: final result
                 const int64_t row = (int64_t)b * p.H_q + g * kG + h;
-                p.out[row * kD + dim] = L > 0.f ? O * kInvPScale / L : 0.f;
+                p.out[row * kD + dim] = L > 0.f ? O / L : 0.f;
                 if (dim == 0) p.lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
             } else {
                 float* part = p.partial + ((int64_t)(blockIdx.x + u) * kG + h) * kPartStride;
@@ -867,7 +898,7 @@ __global__ void __launch_bounds__(kG * kD) merge_kernel(DecodeParams p)
             O += part[4 + dim] * sc;
         }
     }
-    p.out[row * kD + dim] = L > 0.f ? O * kInvPScale / L : 0.f;
+    p.out[row * kD + dim] = L > 0.f ? O / L : 0.f;
     if (dim == 0) p.lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
 }
 

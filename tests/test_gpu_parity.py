@@ -139,6 +139,35 @@ def test_decode_reads_oracle_pages():
         assert_close(out[b, 4 * g:4 * g + 4], lse[b, 4 * g:4 * g + 4], ro[i], rl[i], f"unit {(b, g)}")
 
 
+def test_large_value_scales():
+    """Tokens whose value scales are far above 16 (|v| up to ~1e5): p * vscale
+    * 2^12 would leave the f16 range of the tensor-core weights, so the decode
+    lowers its weight scale; the result stays within tolerance of the oracle."""
+    from compressed_paged_kv_ada_b200 import PagedCache
+
+    w = W.make("ragged64", seq_lens=[700, 33, 1200], H_kv=2, H_q=8)
+    K, V = w.dense(w.seq_lens)
+    rng = np.random.default_rng(11)
+    big = rng.random(len(V)) < 0.05
+    V = V.astype(np.float64) * np.where(big, rng.choice([300.0, 3000.0, 30000.0], len(V)), 1.0)[:, None, None]
+    seq, pos = w.token_index(w.seq_lens)
+    table = oracle.build_page_table(w.tiers, (None, None, None))
+    counts = [int((w.tiers == t).sum()) for t in (1, 2, 3)]
+    pools = oracle.encode_cache(K, V, seq, pos, w.page_offsets, table, counts)
+    ref = dict(B=w.B, H_q=w.H_q, H_kv=w.H_kv, page_offsets=w.page_offsets, seq_lens=w.seq_lens,
+               page_table=table, pools=pools)
+    cache = PagedCache(w.page_offsets, w.seq_lens, w.tiers)
+    for t in range(3):
+        cache.pools[t].copy_(to_torch(pools[t]))
+    q = w.queries()
+    out, lse = _decode(cache, q)
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+    units = [(b, g) for b in range(w.B) for g in range(w.H_kv)]
+    ro, rl = oracle.cache_attention(ref, q, units)
+    for i, (b, g) in enumerate(units):
+        assert_close(out[b, 4 * g:4 * g + 4], lse[b, 4 * g:4 * g + 4], ro[i], rl[i], f"unit {(b, g)}")
+
+
 def test_all_dropped_and_q_zero():
     """A unit whose pages are all dropped gives out 0 and lse -inf; q = 0 gives
     the mean of the kept values and lse = ln(#kept)."""
