@@ -72,9 +72,9 @@ constexpr int kPbufFloats = 16 * kG + 2 * kG;   // p*scale per (token, head); al
 // c has the angle of T2 code 2c.
 constexpr int kFoldOff = (kPbufOff + kWarps * kPbufFloats * 4 + 127) / 128 * 128;
 constexpr int kFoldBytes = 16 * 1024;
-// The unit's query for T1 leaves: even dims and odd dims of leaf j = 8s + i in
-// two 1 KB arrays of 16-byte entries (4 heads) at byte 144 s ^ 16 i, so the 8
-// subtree lanes of a token read 8 distinct banks.
+// The unit's query for T1 leaves: (q[2j], q[2j+1]) of leaf j = 8s + i for
+// heads 0, 1 and for heads 2, 3, in two 1 KB arrays of 16-byte entries at
+// byte 144 s ^ 16 i, so the 8 subtree lanes of a token read 8 distinct banks.
 constexpr int kQOff = kFoldOff + kFoldBytes;
 constexpr int kQBytes = 2 * kLeaves * 16;
 constexpr int kBarOff = kQOff + kQBytes;
@@ -361,7 +361,7 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, const uint8_t* sm
     const uint32_t side4 = (uint32_t)(s & 1) << 2, side5 = (uint32_t)((s >> 1) & 1) << 2;
     const uint32_t side6 = (uint32_t)((s >> 2) & 1) << 2;
     const bool b2 = (s >> 2) & 1, b1 = (s >> 1) & 1;
-#pragma unroll 2
+#pragma unroll 1
     for (int pass = 0; pass < 4; ++pass) {
         const int t = pass * 4 + k;
         uint32_t lo[8], uo[8];
@@ -395,22 +395,34 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, const uint8_t* sm
             wl[2 * m + 1] = w1[m] * f.y;
         }
         float acc[kG];
+        if (T == 1) {
+            // (q[2j], q[2j+1]) . (w cos phi, w sin phi) per head as packed
+            // f32x2 multiply-adds; the two halves are added at the end
+            float2 acc2[kG];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if (T == 1) {
+            for (int j = 0; j < 8; ++j) {
                 const float2 f = *(const float2*)(lut + lo[j]);
-                const float kx = wl[j] * f.x, ky = wl[j] * f.y;
-                const float4 ev = *(const float4*)(smem + kQOff + fl[j]);          // q[2j], 4 heads
-                const float4 od = *(const float4*)(smem + kQOff + 1024 + fl[j]);   // q[2j + 1]
-                const float qev[kG] = {ev.x, ev.y, ev.z, ev.w}, qod[kG] = {od.x, od.y, od.z, od.w};
+                const float2 kk = make_float2(wl[j] * f.x, wl[j] * f.y);
+                const float4 qa = *(const float4*)(smem + kQOff + fl[j]);          // heads 0, 1
+                const float4 qb = *(const float4*)(smem + kQOff + 1024 + fl[j]);   // heads 2, 3
+                const float2 qh[kG] = {make_float2(qa.x, qa.y), make_float2(qa.z, qa.w), make_float2(qb.x, qb.y),
+                                       make_float2(qb.z, qb.w)};
 #pragma unroll
-                for (int h = 0; h < kG; ++h) acc[h] = fmaf(qod[h], ky, j == 0 ? qev[h] * kx : fmaf(qev[h], kx, acc[h]));
-            } else {   // leaf terms already folded with the query
-                const float4 F = *(const float4*)(smem + kFold + lo[j]);
-                const float fv[kG] = {F.x, F.y, F.z, F.w};
-#pragma unroll
-                for (int h = 0; h < kG; ++h) acc[h] = j == 0 ? wl[j] * fv[h] : fmaf(wl[j], fv[h], acc[h]);
+                for (int h = 0; h < kG; ++h)
+                    acc2[h] = j == 0 ? __fmul2_rn(qh[h], kk) : __ffma2_rn(qh[h], kk, acc2[h]);
             }
+#pragma unroll
+            for (int h = 0; h < kG; ++h) acc[h] = acc2[h].x + acc2[h].y;
+        } else {   // leaf terms already folded with the query; heads in f32x2 pairs
+            float2 a01, a23;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float4 F = *(const float4*)(smem + kFold + lo[j]);
+                const float2 ww = make_float2(wl[j], wl[j]);
+                a01 = j == 0 ? __fmul2_rn(ww, make_float2(F.x, F.y)) : __ffma2_rn(ww, make_float2(F.x, F.y), a01);
+                a23 = j == 0 ? __fmul2_rn(ww, make_float2(F.z, F.w)) : __ffma2_rn(ww, make_float2(F.z, F.w), a23);
+            }
+            acc[0] = a01.x; acc[1] = a01.y; acc[2] = a23.x; acc[3] = a23.y;
         }
         // sum over the token's 8 subtrees; lanes s, s^1 end with head 2 b2 + b1
         const float x0 = (b2 ? acc[2] : acc[0]) + __shfl_xor_sync(full, b2 ? acc[0] : acc[2], 4);
@@ -677,11 +689,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
             *(float4*)(smem + kFoldOff + off) = make_float4(v[0], v[1], v[2], v[3]);
         }
         for (int e = tid; e < 2 * kLeaves; e += kThreads) {   // q for T1 leaves
-            const int odd = e >= kLeaves, j = e & 63, sj = j >> 3, ij = j & 7;
-            float v[kG];
-#pragma unroll
-            for (int h = 0; h < kG; ++h) v[h] = p.q[((int64_t)b * p.H_q + g * kG + h) * kD + 2 * j + odd];
-            *(float4*)(smem + kQOff + 1024 * odd + ((144 * sj) ^ (16 * ij))) = make_float4(v[0], v[1], v[2], v[3]);
+            const int half = e >= kLeaves, j = e & 63, sj = j >> 3, ij = j & 7;
+            const float* q0 = p.q + ((int64_t)b * p.H_q + g * kG + 2 * half) * kD + 2 * j;
+            const float* q1 = q0 + kD;
+            *(float4*)(smem + kQOff + 1024 * half + ((144 * sj) ^ (16 * ij))) = make_float4(q0[0], q0[1], q1[0], q1[1]);
         }
         __syncthreads();
         int32_t ra, rb;   // this warp's unit-local page range
