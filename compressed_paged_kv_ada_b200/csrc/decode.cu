@@ -1,40 +1,44 @@
 // decode.cu -- angle-domain attention (ADA) decode over the paged cache.
 //
-// Spherical KV (arXiv 2605.18856), Abstract: logits come "directly from these
-// codes without reconstructing dense keys", on "a paged, block-local,
-// fusion-friendly decode path" that "directly targets HBM traffic".  The logit
-// of query q against a stored key is r * S_root / sqrt(d), with S evaluated
-// bottom-up over the recursive-polar tree:
+// Spherical KV (arXiv 2605.18856), Abstract: the logits are computed from the
+// angle codes themselves, never from rebuilt dense keys, on a paged,
+// block-local decode path whose aim is less HBM traffic.  The logit of query q
+// against a stored key is r * S_root / sqrt(d), with S defined bottom-up over
+// the recursive-polar tree:
 //   leaf j:     S = q[2j] cos(phi_j) + q[2j+1] sin(phi_j)
-//   upper node: S = cos(psi) S_left + sin(psi) S_right.
+//   upper node: S = cos(psi) S_left + sin(psi) S_right
+// and evaluated here in its unrolled (top-down) form.
 // Values are dequantised (int8/int4 code times the token's fp16 scale) inside
 // the value FMA; an online softmax keeps (max, sum, out) per query head, and
 // long contexts are split across SMs and merged with a log-sum-exp combine.
 //
-// Launch structure (three kernels on the caller's stream):
+// Launch structure (three kernels on the caller's stream; decode and merge
+// are programmatic dependent launches that overlap the previous kernel's
+// tail and wait for its results):
 //   plan   -- 1 CTA: unit_start[u] = pages before unit u = (b, g), u = b*H_kv+g.
 //   decode -- persistent, one 512-thread CTA per SM.  The flattened page range
 //             [0, P) is cut into n_cta equal pieces; a CTA walks the units its
-//             piece overlaps.  Its 16 warps take the unit's pages round robin;
-//             each warp bulk-copies a page (cp.async.bulk, mbarrier completion)
-//             into a 2-stage ring in shared memory while it computes the
-//             previous one.
-//             Logits: 4 tokens per pass, 8 lanes per token; lane s owns the
-//             8-leaf subtree s (one aligned code block) and all 4 query heads,
-//             so each table lookup serves 4 heads.  The three top tree levels
-//             use shuffles that leave each lane a different head.  Cos/sin
-//             tables sit in shared memory with 16 lane replicas per code, so a
-//             half warp's 64-bit lookups never share a bank.  T2/T3 leaves
-//             (16 and 8 codes) instead index per-unit tables that already hold
-//             q[2j] cos(phi) + q[2j+1] sin(phi) for the 4 heads: one 16-byte
-//             lookup and no arithmetic per leaf.  (Packed f32x2 arithmetic in
-//             the upper levels would need {cos,cos} and {sin,sin} pairs, i.e.
+//             piece overlaps.  Its 16 warps split each unit's pages into
+//             contiguous ranges of equal tier weight; each warp bulk-copies a
+//             page (cp.async.bulk, mbarrier completion) into a 2-stage ring in
+//             shared memory while it computes the previous one.
+//             Logits, top down: 8 tokens per pass, 4 lanes per token; lane q
+//             owns subtree blocks 2q, 2q+1 (one level-4 node) for all 4 query
+//             heads, so each table lookup serves 4 heads.  The top codes come
+//             by shuffles, and a two-stage butterfly leaves each lane one head.
+//             Cos/sin tables sit in shared memory with 16 lane replicas per
+//             code, so a half warp's 64-bit lookups never share a bank.  T2/T3
+//             leaves (16 and 8 codes) instead index a per-unit table that
+//             already holds q[2j] cos(phi) + q[2j+1] sin(phi) for the 4 heads:
+//             one 16-byte lookup per leaf.  (Packed f32x2 arithmetic in the
+//             upper levels would need {cos,cos} and {sin,sin} pairs, i.e.
 //             16-byte lookups; measured on B200 that doubles shared-memory
 //             traffic and is slower.)
 //             Values: out^T[dims x heads] += V^T[dims x 16 tokens] P^T[16 x 4]
 //             on the tensor cores (mma.sync m16n8k16, f16 operands, fp32
-//             accumulators).  Value codes are exact in f16; the weights p*scale
-//             are split into f16 hi + lo parts (two MMAs), keeping ~22 bits.
+//             accumulators).  Value codes are exact in f16; the weights
+//             p * vscale * sc are split into f16 hi + lo parts (two MMAs),
+//             keeping ~22 bits.
 //   merge  -- one CTA per unit whose pages were split over several CTAs.
 #include <mutex>
 
@@ -176,6 +180,9 @@ __device__ inline bool mbar_wait(uint32_t bar, uint32_t parity)
 // ---------------------------------------------------------------- plan --
 __global__ void __launch_bounds__(1024) plan_kernel(DecodeParams p)
 {
+    // let the decode kernel start its prologue now; it waits for this grid's
+    // results before it reads them
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ int32_t warp_tot[32];
     __shared__ int32_t carry;
     int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -334,102 +341,138 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Table offset of upper code 7 (the block's top node) of one subtree block.
+template <int T>
+__device__ __forceinline__ uint32_t block_top(const uint8_t* codes, int blk, uint32_t base_rep)
+{
+    if (T == 1) return __byte_perm(*(const uint32_t*)(codes + blk * 16 + 12), base_rep, 0x7634);
+    if (T == 2) return ((*(const uint16_t*)(codes + kP * 64 + blk * 2) >> 3) & (63u << 7)) | base_rep;
+    return (((*(const uint32_t*)(codes + blk * 4)) >> 28) << 7) | base_rep;
+}
+
+// One subtree block of a token, top down from its weight v (the product of
+// the radius, the logit scale and the factors of its three ancestors):
+// accumulates the block's per-head sums (T1 in f32x2 (even, odd) pairs,
+// T2/T3 in f32x2 head pairs).
+template <int T>
+__device__ __forceinline__ void subtree(float v, const uint32_t (&lo)[8], const uint32_t (&uo)[8],
+                                        const uint8_t* smem, const uint8_t* lut, const uint8_t* lut_up,
+                                        const uint32_t (&fl)[8], float2 (&acc2)[kG], bool first)
+{
+    float w2[2], w1[4], wl[8];
+    {
+        const float2 f = *(const float2*)(lut_up + uo[6]);
+        w2[0] = v * f.x;
+        w2[1] = v * f.y;
+    }
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+        const float2 f = *(const float2*)(lut_up + uo[4 + n]);
+        w1[2 * n] = w2[n] * f.x;
+        w1[2 * n + 1] = w2[n] * f.y;
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const float2 f = *(const float2*)(lut_up + uo[m]);
+        wl[2 * m] = w1[m] * f.x;
+        wl[2 * m + 1] = w1[m] * f.y;
+    }
+    if (T == 1) {   // (q[2j], q[2j+1]) . (w cos phi, w sin phi) per head
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float2 f = *(const float2*)(lut + lo[j]);
+            const float2 kk = make_float2(wl[j] * f.x, wl[j] * f.y);
+            const float4 qa = *(const float4*)(smem + kQOff + fl[j]);          // heads 0, 1
+            const float4 qb = *(const float4*)(smem + kQOff + 1024 + fl[j]);   // heads 2, 3
+            const float2 qh[kG] = {make_float2(qa.x, qa.y), make_float2(qa.z, qa.w), make_float2(qb.x, qb.y),
+                                   make_float2(qb.z, qb.w)};
+#pragma unroll
+            for (int h = 0; h < kG; ++h)
+                acc2[h] = (first && j == 0) ? __fmul2_rn(qh[h], kk) : __ffma2_rn(qh[h], kk, acc2[h]);
+        }
+    } else {   // leaf terms already folded with the query
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 F = *(const float4*)(smem + kFoldOff + lo[j]);
+            const float2 ww = make_float2(wl[j], wl[j]);
+            acc2[0] = (first && j == 0) ? __fmul2_rn(ww, make_float2(F.x, F.y))
+                                        : __ffma2_rn(ww, make_float2(F.x, F.y), acc2[0]);
+            acc2[1] = (first && j == 0) ? __fmul2_rn(ww, make_float2(F.z, F.w))
+                                        : __ffma2_rn(ww, make_float2(F.z, F.w), acc2[1]);
+        }
+    }
+}
+
 // Logits of the 16 tokens of one page of tier T staged at `pg`, written in the
-// log2 domain to pbuf[t * kG + head].  Lane
-// (k, s) handles subtree s of tokens 4 pass + k for all 4 heads, top down:
-// the tree's value r S_root is the sum over leaves of (product of the factors
-// on the leaf's path: cos(psi) into a left child, sin(psi) into a right one)
-// times the leaf term q[2j] cos(phi_j) + q[2j+1] sin(phi_j).  The path
-// products do not depend on the head, so the per-head work is one
-// multiply-add per leaf (T2/T3, whose leaf terms are read from the
-// query-folded tables) or per dimension (T1).
+// log2 domain to pbuf[t * kG + head].  Lane (k8, q), q = lane & 3, handles
+// the two subtree blocks 2q, 2q+1 (the subtree of level-4 node q) of tokens
+// 8 pass + k8 for all 4 heads, top down: the tree's value r S_root is the sum
+// over leaves of (product of the factors on the leaf's path: cos(psi) into a
+// left child, sin(psi) into a right one) times the leaf term q[2j] cos(phi_j)
+// + q[2j+1] sin(phi_j).  The path products do not depend on the head, so the
+// per-head work is one multiply-add per leaf (T2/T3, whose leaf terms are read
+// from the query-folded table) or per dimension (T1).  Odd tokens take block
+// 2q+1 first, so the 8 lanes of a quarter warp read 8 different subtrees'
+// table rows (8 distinct banks).
 template <int T>
 __device__ __forceinline__ void page_logits(const uint8_t* pg, const uint8_t* smem, float* pbuf, int lane,
-                                            const uint32_t (&fl)[8])
+                                            const uint32_t (&flA)[8])
 {
     const unsigned full = 0xffffffffu;
-    const int k = lane >> 3, s = lane & 7;
+    const int q = lane & 3, k8 = lane >> 2;
+    const bool a_right = k8 & 1;            // block A = 2q + 1 (right child of level-4 node q)
+    const int sA = 2 * q + (k8 & 1), sB = sA ^ 1;
     constexpr int kBase = T == 1 ? kLutT1 : T == 2 ? kLutT2 : kLutT3;
     constexpr int kUp = T == 1 ? 128 : 0;   // upper (cos, sin) inside a row
-    constexpr int kFold = kFoldOff;
     const uint8_t* lut = smem + kBase;
     const uint8_t* lut_up = lut + kUp;
     const uint32_t rep = (uint32_t)(lane & 15) << 3;
     const uint8_t* codes = pg + Tier<1>::f.off_codes;
-    // ancestors of subtree s: level-4 node s>>1, level-5 node s>>2, the root;
-    // the subtree lies on their right (sin, byte 4 of the entry) or left side
-    const uint32_t side4 = (uint32_t)(s & 1) << 2, side5 = (uint32_t)((s >> 1) & 1) << 2;
-    const uint32_t side6 = (uint32_t)((s >> 2) & 1) << 2;
-    const bool b2 = (s >> 2) & 1, b1 = (s >> 1) & 1;
+    uint32_t flB[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) flB[i] = flA[i] ^ 144u;   // 144 sB ^ 16 i
+    // ancestors: the root (level-5 node q>>1 is its left child for q < 2) and
+    // level-5 node q>>1 (level-4 node q is its left child for even q)
+    const uint32_t side6 = (uint32_t)(q >> 1) << 2, side5 = (uint32_t)(q & 1) << 2;
+    const int base = lane & ~3;
 #pragma unroll 1
-    for (int pass = 0; pass < 4; ++pass) {
-        const int t = pass * 4 + k;
+    for (int pass = 0; pass < 2; ++pass) {
+        const int t = pass * 8 + k8;
         uint32_t lo[8], uo[8];
-        block_offsets<T>(codes, t * 8 + s, rep, fl, lo, uo);
-        // top codes: block i carries top node i (level 4 nodes 0..3, level 5
-        // nodes 0..1, root)
-        const uint32_t o4 = __shfl_sync(full, uo[7], (lane & ~7) | (s >> 1));
-        const uint32_t o5 = __shfl_sync(full, uo[7], (lane & ~7) | (4 + (s >> 2)));
-        const uint32_t o6 = __shfl_sync(full, uo[7], (lane & ~7) | 6);
+        block_offsets<T>(codes, t * 8 + sA, rep, flA, lo, uo);
+        const uint32_t topB = block_top<T>(codes, t * 8 + sB, rep);
+        // top codes: block i's slot 7 is top node i (level-4 nodes 0..3,
+        // level-5 nodes 0..1, root).  This lane has those of blocks 2q, 2q+1,
+        // as two 16-bit table offsets.
+        const uint32_t top2 = (a_right ? topB : uo[7]) | ((a_right ? uo[7] : topB) << 16);
+        const uint32_t w4 = __shfl_sync(full, top2, base + (q >> 1));   // block q
+        const uint32_t w5 = __shfl_sync(full, top2, base + 2);          // block 4 + (q >> 1)
+        const uint32_t w6 = __shfl_sync(full, top2, base + 3);          // block 6
+        const uint32_t o4 = (w4 >> (16 * (q & 1))) & 0xffffu;
+        const uint32_t o5 = (w5 >> (16 * (q >> 1))) & 0xffffu;
+        const uint32_t o6 = w6 & 0xffffu;
         float v = __half2float(((const __half*)pg)[t]) * kLogitScale;
         v *= *(const float*)(lut_up + o6 + side6);
         v *= *(const float*)(lut_up + o5 + side5);
-        v *= *(const float*)(lut_up + o4 + side4);
-        // level 3 (subtree root, code 6), level 2 (codes 4, 5), level 1 (codes 0..3)
-        float w2[2], w1[4], wl[8];
-        {
-            const float2 f = *(const float2*)(lut_up + uo[6]);
-            w2[0] = v * f.x;
-            w2[1] = v * f.y;
-        }
-#pragma unroll
-        for (int n = 0; n < 2; ++n) {
-            const float2 f = *(const float2*)(lut_up + uo[4 + n]);
-            w1[2 * n] = w2[n] * f.x;
-            w1[2 * n + 1] = w2[n] * f.y;
-        }
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const float2 f = *(const float2*)(lut_up + uo[m]);
-            wl[2 * m] = w1[m] * f.x;
-            wl[2 * m + 1] = w1[m] * f.y;
-        }
+        const float2 f4 = *(const float2*)(lut_up + o4);
+        const float vA = v * (a_right ? f4.y : f4.x), vB = v * (a_right ? f4.x : f4.y);
+        float2 acc2[kG];
+        subtree<T>(vA, lo, uo, smem, lut, lut_up, flA, acc2, true);
+        block_offsets<T>(codes, t * 8 + sB, rep, flB, lo, uo);
+        subtree<T>(vB, lo, uo, smem, lut, lut_up, flB, acc2, false);
         float acc[kG];
         if (T == 1) {
-            // (q[2j], q[2j+1]) . (w cos phi, w sin phi) per head as packed
-            // f32x2 multiply-adds; the two halves are added at the end
-            float2 acc2[kG];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float2 f = *(const float2*)(lut + lo[j]);
-                const float2 kk = make_float2(wl[j] * f.x, wl[j] * f.y);
-                const float4 qa = *(const float4*)(smem + kQOff + fl[j]);          // heads 0, 1
-                const float4 qb = *(const float4*)(smem + kQOff + 1024 + fl[j]);   // heads 2, 3
-                const float2 qh[kG] = {make_float2(qa.x, qa.y), make_float2(qa.z, qa.w), make_float2(qb.x, qb.y),
-                                       make_float2(qb.z, qb.w)};
-#pragma unroll
-                for (int h = 0; h < kG; ++h)
-                    acc2[h] = j == 0 ? __fmul2_rn(qh[h], kk) : __ffma2_rn(qh[h], kk, acc2[h]);
-            }
 #pragma unroll
             for (int h = 0; h < kG; ++h) acc[h] = acc2[h].x + acc2[h].y;
-        } else {   // leaf terms already folded with the query; heads in f32x2 pairs
-            float2 a01, a23;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float4 F = *(const float4*)(smem + kFold + lo[j]);
-                const float2 ww = make_float2(wl[j], wl[j]);
-                a01 = j == 0 ? __fmul2_rn(ww, make_float2(F.x, F.y)) : __ffma2_rn(ww, make_float2(F.x, F.y), a01);
-                a23 = j == 0 ? __fmul2_rn(ww, make_float2(F.z, F.w)) : __ffma2_rn(ww, make_float2(F.z, F.w), a23);
-            }
-            acc[0] = a01.x; acc[1] = a01.y; acc[2] = a23.x; acc[3] = a23.y;
+        } else {
+            acc[0] = acc2[0].x; acc[1] = acc2[0].y; acc[2] = acc2[1].x; acc[3] = acc2[1].y;
         }
-        // sum over the token's 8 subtrees; lanes s, s^1 end with head 2 b2 + b1
-        const float x0 = (b2 ? acc[2] : acc[0]) + __shfl_xor_sync(full, b2 ? acc[0] : acc[2], 4);
-        const float x1 = (b2 ? acc[3] : acc[1]) + __shfl_xor_sync(full, b2 ? acc[1] : acc[3], 4);
-        float y = (b1 ? x1 : x0) + __shfl_xor_sync(full, b1 ? x0 : x1, 2);
-        y += __shfl_xor_sync(full, y, 1);
-        if (!(s & 1)) pbuf[t * kG + 2 * b2 + b1] = y;
+        // sum over the token's 4 lanes; lane q ends with head q
+        const bool b1 = q >> 1, b0 = q & 1;
+        const float x0 = (b1 ? acc[2] : acc[0]) + __shfl_xor_sync(full, b1 ? acc[0] : acc[2], 2);
+        const float x1 = (b1 ? acc[3] : acc[1]) + __shfl_xor_sync(full, b1 ? acc[1] : acc[3], 2);
+        const float y = (b0 ? x1 : x0) + __shfl_xor_sync(full, b0 ? x0 : x1, 1);
+        pbuf[t * kG + q] = y;
     }
 }
 
@@ -630,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
     // and the T1 query arrays
     uint32_t fl[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) fl[i] = (144u * (uint32_t)(lane & 7)) ^ (16u * i);
+    for (int i = 0; i < 8; ++i) fl[i] = (144u * (uint32_t)(2 * (lane & 3) + ((lane >> 2) & 1))) ^ (16u * i);
     uint8_t* stage = smem + kStageOff + w * kStages * kStageBytes;
     float* pbuf = (float*)(smem + kPbufOff) + w * kPbufFloats;
     const uint32_t bar0 = smem_u32(smem + kBarOff + w * kStages * 8);
@@ -641,6 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
     }
     __syncthreads();
 
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // plan_kernel's results are visible
     const int32_t P = p.unit_start[p.n_units];
     const int32_t lo = cta_bound(blockIdx.x, P, p.n_cta), hi = cta_bound(blockIdx.x + 1, P, p.n_cta);
     uint32_t phase = 0;   // bit s = parity to wait for on stage s
@@ -875,6 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
 // --------------------------------------------------------------- merge --
 __global__ void __launch_bounds__(kG * kD) merge_kernel(DecodeParams p)
 {
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // decode_kernel's partials are visible
     const int u = blockIdx.x;
     const int h = threadIdx.x >> 7, dim = threadIdx.x & (kD - 1);
     const int32_t P = p.unit_start[p.n_units];
@@ -911,6 +956,30 @@ __global__ void __launch_bounds__(kG * kD) merge_kernel(DecodeParams p)
     }
     p.out[row * kD + dim] = L > 0.f ? O / L : 0.f;
     if (dim == 0) p.lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+}
+
+// plan, decode, merge on stream s.  decode and merge are launched as
+// programmatic dependents (PDL): each may start its prologue while the kernel
+// before it finishes, and waits (griddepcontrol.wait) before reading that
+// kernel's results.
+void launch_decode(const DecodeParams& p, cudaStream_t s)
+{
+    plan_kernel<<<1, 1024, 0, s>>>(p);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(p.n_cta);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, decode_kernel, p);
+    cfg.gridDim = dim3(p.n_units);
+    cfg.blockDim = dim3(kG * kD);
+    cfg.dynamicSmemBytes = 0;
+    cudaLaunchKernelEx(&cfg, merge_kernel, p);
 }
 
 int sm_count(int n_sm)
@@ -1023,9 +1092,7 @@ extern "C" sphkv_status sphkv_decode_attention(const sphkv_cache* c, int32_t H_q
         attr_dev = dev;
     }
     cudaStream_t s = (cudaStream_t)stream;
-    plan_kernel<<<1, 1024, 0, s>>>(p);
-    decode_kernel<<<p.n_cta, kThreads, kSmemBytes, s>>>(p);
-    merge_kernel<<<p.n_units, kG * kD, 0, s>>>(p);
+    launch_decode(p, s);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) {
         sphkv_set_error("sphkv_decode_attention: launch failed: %s", cudaGetErrorString(err));
@@ -1139,9 +1206,7 @@ extern "C" sphkv_status sphkv_decode_attention_noalloc(const sphkv_cache* c, int
     p.partial = (float*)((uint8_t*)scratch + part_off);
     p.status = status_dev;
     cudaStream_t s = (cudaStream_t)stream;
-    plan_kernel<<<1, 1024, 0, s>>>(p);
-    decode_kernel<<<p.n_cta, kThreads, kSmemBytes, s>>>(p);
-    merge_kernel<<<p.n_units, kG * kD, 0, s>>>(p);
+    launch_decode(p, s);
     const cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) {
         sphkv_set_error("sphkv_decode_attention_noalloc: launch failed: %s", cudaGetErrorString(err));
