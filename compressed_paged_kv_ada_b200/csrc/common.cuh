@@ -2,9 +2,9 @@
 // kernels (encode, RDR, page table, decode).  Nothing here is used by, or
 // uses, the CPU oracle.
 //
-// Page format (Spherical KV, arXiv 2605.18856, Abstract: "tier-homogeneous
-// pages with lightweight metadata and coalesced reads"; the byte layout is
-// this library's, described in include/sphkv.h):
+// Page format (Spherical KV, arXiv 2605.18856, Abstract: every page holds
+// one tier, carries little metadata and is read contiguously; the byte layout
+// is this library's, described in include/sphkv.h):
 //   r[16] fp16 | vscale[16] fp16 | code planes (8 subtree blocks per token)
 //   | value rows (channels permuted for tensor-core fragments)
 #pragma once

@@ -1,8 +1,7 @@
 // encode.cu -- dense K/V rows -> tier pages (prefill and append).
 //
-// Spherical KV (arXiv 2605.18856), Abstract: ADA stores each key "in a
-// spherical parameterization consisting of a scalar radius and compact angle
-// codes".  The recursive-polar tree, grids and bit layout are this library's
+// Spherical KV (arXiv 2605.18856), Abstract: ADA keeps each key in spherical
+// form, as a radius and a set of compact angle codes.  The recursive-polar tree, grids and bit layout are this library's
 // fixed format (see include/sphkv.h).
 //
 // One warp per (token, kv head).  Lane l owns dims 4l..4l+3, i.e. leaves 2l and

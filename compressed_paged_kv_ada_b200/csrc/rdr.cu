@@ -1,10 +1,10 @@
 // rdr.cu -- rate-distortion retention (RDR) tier assignment and page-table
 // construction.
 //
-// Spherical KV (arXiv 2605.18856), Abstract: RDR "treats KV allocation as a
-// rate-distortion problem" and "jointly chooses keep/drop decisions and
-// precision tiers per token and head under a fixed budget, producing
-// tier-homogeneous pages with lightweight metadata".  This library's reading:
+// Spherical KV (arXiv 2605.18856), Abstract: RDR casts the allocation of KV
+// storage as a rate-distortion trade-off, picking keep/drop and a precision
+// tier together under a fixed budget, and the result is pages that each hold
+// one tier with little metadata.  This library's reading:
 // the unit is a 16-token page of one kv head; rate = page bytes of the tier,
 // distortion = page utility x eps[tier]; a Lagrangian argmin with lambda found
 // by doubling then 100 bisection steps, always keeping the feasible end.

@@ -119,7 +119,7 @@ const char* sphkv_last_error(void);
 
 /*
  * sphkv_encode -- dense K/V rows -> tier pages (prefill and append).
- *   Spherical KV Abstract (ADA: "a scalar radius and compact angle codes").
+ *   Spherical KV, Abstract (ADA: a key becomes a radius plus angle codes).
  *   K, V: [n_tok][H_kv][128], dtype SPHKV_DTYPE_BF16 or SPHKV_DTYPE_F32.
  *   tok_seq, tok_pos: [n_tok] int32, sequence and position of each row.
  *   For each row and kv head the page-table entry of (seq, pos / 16) picks the
@@ -137,9 +137,9 @@ sphkv_status sphkv_encode(const sphkv_cache* cache, const void* K, const void* V
 
 /*
  * sphkv_rdr_workspace_bytes / sphkv_rdr_assign -- rate-distortion retention.
- *   Spherical KV Abstract (RDR: keep/drop and precision tiers "under a fixed
- *   budget", "a rate-distortion problem"); the Lagrangian form is this
- *   library's reading.  Units are (kv head g, sequence b, page p) for
+ *   Spherical KV, Abstract (RDR: keep/drop and precision tiers chosen under
+ *   a fixed byte budget as a rate-distortion trade-off); the Lagrangian form
+ *   is this library's reading.  Units are (kv head g, sequence b, page p) for
  *   p < ceil(seq_len[b] / 16).  Page utility U = sum of `utility` over the
  *   page's present tokens, summed in slot order in fp64.  Rate R = page bytes
  *   of the tier (drop 0), distortion D = U * eps[tier].  The first n_sink and
@@ -167,8 +167,8 @@ sphkv_status sphkv_rdr_assign(const sphkv_cache* cache, const float* utility, co
 
 /*
  * sphkv_build_page_table -- tiers -> page-table entries.
- *   Spherical KV Abstract ("tier-homogeneous pages with lightweight
- *   metadata").  tiers: [n_entries] uint8 (0 drop, 1..3) in table order; the
+ *   Spherical KV, Abstract (each page holds one tier, with little metadata
+ *   per page).  tiers: [n_entries] uint8 (0 drop, 1..3) in table order; the
  *   k-th entry of tier t (in table order) gets pool page perm_t[k], or k when
  *   perm_t is NULL.  table: [n_entries] int32 out.  counts_out: device int64[3]
  *   pages used per tier (may be NULL).  One kernel, a block-wide scan.
@@ -180,9 +180,9 @@ sphkv_status sphkv_build_page_table(const uint8_t* tiers, int64_t n_entries, con
 
 /*
  * sphkv_decode_workspace_bytes / sphkv_decode_attention -- ADA decode.
- *   Spherical KV Abstract ("computes attention logits directly from these
- *   codes without reconstructing dense keys"; "a paged, block-local,
- *   fusion-friendly decode path").  One decode query per sequence.
+ *   Spherical KV, Abstract (logits come from the codes themselves, no dense
+ *   key is rebuilt, over paged block-local storage).  One decode query per
+ *   sequence.
  *   q: [B][H_q][128] fp32.  out: [B][H_q][128] fp32 = softmax-weighted sum of
  *   the dequantised values of the kept tokens (t < seq_len, page not dropped);
  *   lse: [B][H_q] fp32, natural-log log-sum-exp of the logits (scale 1/sqrt(d)

@@ -18,8 +18,8 @@
  * here is the one this project fixes: a recursive-polar (binary-tree)
  * parameterisation with d/2 leaf pair angles and d/2-1 upper angles, three
  * tiers (T1 8/8 bits + int8 V, T2 4/6 bits + int4 V, T3 3/4 bits + int4 V),
- * 16-token pages and a Lagrangian bisection for RDR.  Every reading of a point
- * the pages leave open is listed in the project's design notes.
+ * 16-token pages and a Lagrangian bisection for RDR.  Where the pages leave a
+ * point open, the reading taken is stated next to the code that takes it.
  *
  * How.  Plain loops in fp64, compiled with -ffp-contract=off so no product is
  * ever fused into an add.  Attention is done the slow, obvious way: decode the
