@@ -287,16 +287,27 @@ def run_gpu(args):
                      torch.arange(n, dtype=torch.int32, device=dev))
         del Kt, Vt
     cache.check()
-    q_np = w.queries()
-    q = torch.from_numpy(q_np).to(dev)
-    out = torch.empty((w.B, w.H_q, 128), dtype=torch.float32, device=dev)
-    lse = torch.empty((w.B, w.H_q), dtype=torch.float32, device=dev)
-    ws = cache.workspace(w.H_q)
+    n_q = args.n_q
     desc = cache.descriptor()
     stream = torch.cuda.current_stream(dev)
+    if n_q == 1:
+        q_np = w.queries()
+        out = torch.empty((w.B, w.H_q, 128), dtype=torch.float32, device=dev)
+        lse = torch.empty((w.B, w.H_q), dtype=torch.float32, device=dev)
+        ws = cache.workspace(w.H_q)
+    else:   # n_q causal query tokens per sequence (seeded as decode steps 0 .. n_q-1)
+        q_np = np.stack([w.queries(step=i) for i in range(n_q)], axis=1)
+        out = torch.empty((w.B, n_q, w.H_q, 128), dtype=torch.float32, device=dev)
+        lse = torch.empty((w.B, n_q, w.H_q), dtype=torch.float32, device=dev)
+        ws = torch.empty(L.sphkv_decode_mq_workspace_bytes(w.B, w.H_q, w.H_kv, w.total_pages), dtype=torch.uint8,
+                         device=dev)
+    q = torch.from_numpy(q_np).to(dev)
 
     def step():
-        L.sphkv_decode_attention(desc, w.H_q, q, out, lse, ws, status=cache.status, stream=stream)
+        if n_q == 1:
+            L.sphkv_decode_attention(desc, w.H_q, q, out, lse, ws, status=cache.status, stream=stream)
+        else:
+            L.sphkv_decode_attention_mq(desc, n_q, w.H_q, q, out, lse, ws, status=cache.status, stream=stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -326,7 +337,8 @@ def run_gpu(args):
     ms_total = start.elapsed_time(end)
     call_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
     ms_step = ms_total / args.steps
-    units = int(w.seq_lens.sum()) * w.H_q
+    # token-heads served: query token i attends to seq_len - (n_q - 1 - i) tokens
+    units = int(sum(np.maximum(w.seq_lens - (n_q - 1 - i), 0).sum() for i in range(n_q))) * w.H_q
     t_all = [ms_step]
     u_all = [units]
     if world > 1:
@@ -358,17 +370,20 @@ def run_gpu(args):
 
     line = None
     if rank == 0:
-        algo = algorithmic_bytes(w)
+        # the cache once per step, plus the extra query tokens' q, out and lse
+        algo = algorithmic_bytes(w) + (n_q - 1) * w.B * w.H_q * (128 * 4 * 2 + 4)
         peak, peak_kind = measured_peaks()
         achieved = algo / (call_ms / 1e3) / 1e9
         traffic = profiled_traffic(os.path.join(ROOT, "compressed_paged_kv_ada_b200", "csrc", "decode.cu"),
-                                   os.path.join(ROOT, "profiles", "decode_kernel_llama32k.md"))
-        cb = cpu_baseline(w, q_np, budget_s=args.cpu_seconds) if (world == 1 and args.cpu_seconds > 0) else None
+                                   os.path.join(ROOT, "profiles", "decode_kernel_llama32k.md")) if n_q == 1 else None
+        cb = (cpu_baseline(w, q_np, budget_s=args.cpu_seconds)
+              if (world == 1 and args.cpu_seconds > 0 and n_q == 1) else None)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": WORKLOAD_DESC, "global_batch": w.B * world, "seq_len": int(w.seq_lens[0]),
+            "config": {"workload": WORKLOAD_DESC + (f"; {n_q} causal query tokens per sequence" if n_q > 1 else ""),
+                       "n_q": n_q, "global_batch": w.B * world, "seq_len": int(w.seq_lens[0]),
                        "parallelism": f"replicas x{world} (batch sharded, no exchange)",
                        "l2": "compressed cache per step larger than L2 (126 MB); no flush",
                        "algorithmic_bytes_per_step": algo,
@@ -376,12 +391,13 @@ def run_gpu(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_kind} hbm_gbs (copy, burst)",
-                         "kernel": "sphkv_decode_attention call (plan + decode + merge), per-call CUDA events"},
+                         "kernel": ("sphkv_decode_attention" if n_q == 1 else "sphkv_decode_attention_mq")
+                                   + " call (plan + decode + merge per query pair), per-call CUDA events"},
             "cpu_baseline": cb,
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": int(q.numel() * 4),
                     "d2h_bytes_per_step": int(out.numel() * 4 + lse.numel() * 4)},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": 3 * ((n_q + 1) // 2) * args.steps,
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
@@ -397,6 +413,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--n-q", type=int, default=1,
+                    help="query tokens per sequence and step (causal multi-token decode; 1 = the headline)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="seconds of oracle time for the cpu_baseline field (0 to skip)")
     args = ap.parse_args(argv)

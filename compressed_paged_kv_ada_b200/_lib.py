@@ -44,7 +44,8 @@ class sphkv_cache(ctypes.Structure):
 _lib = None
 _EXPORTS = ("sphkv_page_bytes", "sphkv_last_error", "sphkv_encode", "sphkv_rdr_workspace_bytes",
             "sphkv_rdr_assign", "sphkv_build_page_table", "sphkv_decode_workspace_bytes",
-            "sphkv_decode_attention", "sphkv_decode_attention_noalloc")
+            "sphkv_decode_attention", "sphkv_decode_attention_noalloc", "sphkv_decode_mq_workspace_bytes",
+            "sphkv_decode_attention_mq")
 
 
 def lib() -> ctypes.CDLL:
@@ -75,6 +76,11 @@ def lib() -> ctypes.CDLL:
                                              P, P]
         L.sphkv_decode_attention_noalloc.restype = c.c_int
         L.sphkv_decode_attention_noalloc.argtypes = [c.POINTER(sphkv_cache), c.c_int32, P, P, P, P, P]
+        L.sphkv_decode_mq_workspace_bytes.restype = c.c_size_t
+        L.sphkv_decode_mq_workspace_bytes.argtypes = [c.c_int32, c.c_int32, c.c_int32, c.c_int64, c.c_int32]
+        L.sphkv_decode_attention_mq.restype = c.c_int
+        L.sphkv_decode_attention_mq.argtypes = [c.POINTER(sphkv_cache), c.c_int32, c.c_int32, P, P, P, P,
+                                                c.c_size_t, P, P]
         _lib = L
     return _lib
 
@@ -181,3 +187,18 @@ def sphkv_decode_attention_noalloc(cache: sphkv_cache, H_q: int, q: torch.Tensor
     _check("sphkv_decode_attention_noalloc", lib().sphkv_decode_attention_noalloc(
         ctypes.byref(cache), int(H_q), _ptr(q, torch.float32, "q"), _ptr(out, torch.float32, "out"),
         _ptr(lse, torch.float32, "lse"), _ptr(status, torch.int32, "status"), _stream(stream)))
+
+
+def sphkv_decode_mq_workspace_bytes(B: int, H_q: int, H_kv: int, total_pages: int, n_sm: int = 0) -> int:
+    return int(lib().sphkv_decode_mq_workspace_bytes(B, H_q, H_kv, total_pages, n_sm))
+
+
+def sphkv_decode_attention_mq(cache: sphkv_cache, n_q: int, H_q: int, q: torch.Tensor, out: torch.Tensor,
+                              lse: torch.Tensor, workspace: torch.Tensor,
+                              status: Optional[torch.Tensor] = None, stream=None):
+    """Decode attention for n_q causal query tokens per sequence:
+    q, out [B, n_q, H_q, 128], lse [B, n_q, H_q]."""
+    _check("sphkv_decode_attention_mq", lib().sphkv_decode_attention_mq(
+        ctypes.byref(cache), int(n_q), int(H_q), _ptr(q, torch.float32, "q"), _ptr(out, torch.float32, "out"),
+        _ptr(lse, torch.float32, "lse"), _ptr(workspace, torch.uint8, "workspace"),
+        int(workspace.numel()), _ptr(status, torch.int32, "status"), _stream(stream)))

@@ -71,6 +71,18 @@ class PagedCache:
         L.sphkv_decode_attention(self.descriptor(), H_q, q, out, lse, self.workspace(H_q), status=self.status)
         return out, lse
 
+    def decode_mq(self, q: torch.Tensor, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+        """Decode for n_q causal query tokens per sequence: q [B, n_q, H_q, 128];
+        query token i sees the first seq_len - (n_q - 1 - i) tokens."""
+        B, n_q, H_q, d = q.shape
+        out = torch.empty((B, n_q, H_q, d), dtype=torch.float32, device=self.device) if out is None else out
+        lse = torch.empty((B, n_q, H_q), dtype=torch.float32, device=self.device) if lse is None else lse
+        n = L.sphkv_decode_mq_workspace_bytes(self.B, H_q, self.H_kv, self.total_pages)
+        if self._ws is None or self._ws.numel() < n:
+            self._ws = torch.empty(n, dtype=torch.uint8, device=self.device)
+        L.sphkv_decode_attention_mq(self.descriptor(), n_q, H_q, q, out, lse, self._ws, status=self.status)
+        return out, lse
+
     def rdr_assign(self, utility: torch.Tensor, eps, budget: int, n_sink: int, n_recent: int):
         """Choose tiers by RDR (on the device) and write them into self.tiers.
         Returns (lambda, bytes) as device tensors."""

@@ -111,11 +111,17 @@ struct DecodeParams {
     int64_t pool_pages[4];
     int64_t total_pages;
     int B, H_kv, H_q, n_units, n_cta;
+    // Query tokens per sequence (nq), the first of those this launch handles
+    // (q0) and how many it handles (npair, 1 or 2); query token i sees the
+    // first seq_len - (nq - 1 - i) tokens.  q, out: [B][nq][H_q][128],
+    // lse: [B][nq][H_q].  len_shift = nq - q0 - npair: the launch's page range
+    // is that of its last query token.
+    int nq, q0, npair, len_shift;
     const float* q;
     float* out;
     float* lse;
     int32_t* unit_start;   // [n_units + 1]
-    float* partial;        // [n_cta + n_units][kG][kPartStride]
+    float* partial;        // [n_cta + n_units][heads per unit][kPartStride]
     int32_t* status;
 };
 
@@ -200,10 +206,12 @@ __global__ void __launch_bounds__(1024) plan_kernel(DecodeParams p)
                 cap = 0;
             }
             int64_t len = p.seq_lens[b];
+            if (len < 0) report(p.status, SPHKV_ERR_DATA);
+            len = len - p.len_shift > 0 ? len - p.len_shift : 0;
             int64_t np = (len + kP - 1) / kP;
-            if (len < 0 || np > cap) {
+            if (np > cap) {
                 report(p.status, SPHKV_ERR_DATA);
-                np = len < 0 ? 0 : cap;
+                np = cap;
             }
             n = (int32_t)np;
         }
@@ -476,72 +484,19 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, const uint8_t* sm
     }
 }
 
-// One page of tier `tier` already staged in shared memory at `pg`.  The logits
-// are tier-specialised; the softmax and the value MMAs are one copy of code
-// for all tiers apart from the value conversion.
-__device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int valid, const uint8_t* smem, float* pbuf,
-                                             int lane, const uint32_t (&fl)[8], WarpState& st)
+// Values on the tensor cores for one staged page: out^T[dims x heads] +=
+// V^T[dims x 16 tokens] P^T[16 x GQ heads], with the weights P already in
+// pbuf[t * GQ + head] and the per-head rescale factor at pbuf[16 GQ + head].
+// Thread (g, c): B columns = head g (g < GQ), rows = tokens 2c, 2c+1 (b0) and
+// 2c+8, 2c+9 (b1); accumulator columns = heads 2c, 2c+1 (mod GQ).
+template <int GQ>
+__device__ __forceinline__ void page_values(const uint8_t* pg, int tier, const float* pbuf, int lane, float alpha_acc,
+                                            WarpState& st)
 {
     const unsigned full = 0xffffffffu;
-    const int k = lane >> 3, s = lane & 7;
-    const int head = (s & 1) * 2 + ((s >> 1) & 1);
-    // `valid` waits in the buffer's spare word while the logits hold the registers
-    if (lane == 0) ((int*)pbuf)[16 * kG + kG] = valid;
-    if (tier == 1) page_logits<1>(pg, smem, pbuf, lane, fl);
-    else if (tier == 2) page_logits<2>(pg, smem, pbuf, lane, fl);
-    else page_logits<3>(pg, smem, pbuf, lane, fl);
-    __syncwarp();
-    valid = ((const int*)pbuf)[16 * kG + kG];
-    float lg[4];
-#pragma unroll
-    for (int pass = 0; pass < 4; ++pass)   // slots past `valid` (last page) get -inf
-        lg[pass] = pass * 4 + k < valid ? pbuf[(pass * 4 + k) * kG + head] : -INFINITY;
-    __syncwarp();
-    // online softmax for this lane's head (lanes k = 0..3 share it)
-    float pm = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
-    pm = fmaxf(pm, __shfl_xor_sync(full, pm, 8));
-    pm = fmaxf(pm, __shfl_xor_sync(full, pm, 16));
-    const float m_new = fmaxf(st.m, pm);
-    const float alpha = fast_exp2(st.m - m_new);   // st.m = -inf on the first page -> 0
-    st.m = m_new;
-    const __half* vs = (const __half*)(pg + 2 * kP);
-    float wv[4];   // vscale * sc of this lane's tokens
-    bool big = false;
-#pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-        const int t = pass * 4 + k;   // slots past `valid` may hold stale scales: weight exactly 0
-        wv[pass] = t < valid ? __half2float(vs[t]) * st.sc : 0.f;
-        big |= wv[pass] > kWeightMax;
-    }
-    float alpha_acc = alpha;
-    if (__any_sync(full, big)) {   // rare: lower sc so every weight fits f16
-        float vm = fmaxf(fmaxf(wv[0], wv[1]), fmaxf(wv[2], wv[3]));
-        vm = fmaxf(vm, __shfl_xor_sync(full, vm, 8));
-        vm = fmaxf(vm, __shfl_xor_sync(full, vm, 16));
-        const float ratio = pow2_floor(kWeightMax / vm);   // exact: both powers of two scale exactly
-        st.sc *= ratio;
-        alpha_acc *= ratio;
-#pragma unroll
-        for (int pass = 0; pass < 4; ++pass) wv[pass] *= ratio;
-    }
-    float psum = 0.f;
-#pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-        const float pv = fast_exp2(lg[pass] - m_new);
-        psum += pv;
-        const int t = pass * 4 + k;
-        if (s < 4) pbuf[t * kG + head] = pv * wv[pass];
-    }
-    st.l = st.l * alpha + psum;
-    if (lane < 4) pbuf[16 * kG + head] = alpha_acc;
-    __syncwarp();
-
-    // values on the tensor cores.  Thread (g, c): B columns = head g (g < 4),
-    // rows = tokens 2c, 2c+1 (b0) and 2c+8, 2c+9 (b1); accumulator columns =
-    // heads 2c, 2c+1.
     const int g = lane >> 2, c = lane & 3;
     if (__any_sync(full, alpha_acc != 1.f)) {   // a running max or sc moved: rescale (rare after the first pages)
-        const float2 al = *(const float2*)(pbuf + 16 * kG + 2 * (c & 1));
+        const float2 al = *(const float2*)(pbuf + 16 * GQ + (2 * c) % GQ);
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
             st.acc[m][0] *= al.x;
@@ -551,9 +506,9 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
         }
     }
     uint32_t bh0 = 0, bh1 = 0, bl0 = 0, bl1 = 0;
-    if (g < kG) {
-        const float p0 = pbuf[(2 * c) * kG + g], p1 = pbuf[(2 * c + 1) * kG + g];
-        const float p2 = pbuf[(2 * c + 8) * kG + g], p3 = pbuf[(2 * c + 9) * kG + g];
+    if (g < GQ) {
+        const float p0 = pbuf[(2 * c) * GQ + g], p1 = pbuf[(2 * c + 1) * GQ + g];
+        const float p2 = pbuf[(2 * c + 8) * GQ + g], p3 = pbuf[(2 * c + 9) * GQ + g];
         const __half2 h01 = __floats2half2_rn(p0, p1), h23 = __floats2half2_rn(p2, p3);
         bh0 = *(const uint32_t*)&h01;
         bh1 = *(const uint32_t*)&h23;
@@ -635,12 +590,283 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
             mma_16816(st.acc[m], a, bl0, bl1);
         }
     }
+}
+
+// One page of tier `tier` already staged in shared memory at `pg`.  The logits
+// are tier-specialised; the softmax and the value MMAs are one copy of code
+// for all tiers apart from the value conversion.
+__device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int valid, const uint8_t* smem, float* pbuf,
+                                             int lane, const uint32_t (&fl)[8], WarpState& st)
+{
+    const unsigned full = 0xffffffffu;
+    const int k = lane >> 3, s = lane & 7;
+    const int head = (s & 1) * 2 + ((s >> 1) & 1);
+    // `valid` waits in the buffer's spare word while the logits hold the registers
+    if (lane == 0) ((int*)pbuf)[16 * kG + kG] = valid;
+    if (tier == 1) page_logits<1>(pg, smem, pbuf, lane, fl);
+    else if (tier == 2) page_logits<2>(pg, smem, pbuf, lane, fl);
+    else page_logits<3>(pg, smem, pbuf, lane, fl);
+    __syncwarp();
+    valid = ((const int*)pbuf)[16 * kG + kG];
+    float lg[4];
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass)   // slots past `valid` (last page) get -inf
+        lg[pass] = pass * 4 + k < valid ? pbuf[(pass * 4 + k) * kG + head] : -INFINITY;
+    __syncwarp();
+    // online softmax for this lane's head (lanes k = 0..3 share it)
+    float pm = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
+    pm = fmaxf(pm, __shfl_xor_sync(full, pm, 8));
+    pm = fmaxf(pm, __shfl_xor_sync(full, pm, 16));
+    const float m_new = fmaxf(st.m, pm);
+    const float alpha = fast_exp2(st.m - m_new);   // st.m = -inf on the first page -> 0
+    st.m = m_new;
+    const __half* vs = (const __half*)(pg + 2 * kP);
+    float wv[4];   // vscale * sc of this lane's tokens
+    bool big = false;
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+        const int t = pass * 4 + k;   // slots past `valid` may hold stale scales: weight exactly 0
+        wv[pass] = t < valid ? __half2float(vs[t]) * st.sc : 0.f;
+        big |= wv[pass] > kWeightMax;
+    }
+    float alpha_acc = alpha;
+    if (__any_sync(full, big)) {   // rare: lower sc so every weight fits f16
+        float vm = fmaxf(fmaxf(wv[0], wv[1]), fmaxf(wv[2], wv[3]));
+        vm = fmaxf(vm, __shfl_xor_sync(full, vm, 8));
+        vm = fmaxf(vm, __shfl_xor_sync(full, vm, 16));
+        const float ratio = pow2_floor(kWeightMax / vm);   // exact: both powers of two scale exactly
+        st.sc *= ratio;
+        alpha_acc *= ratio;
+#pragma unroll
+        for (int pass = 0; pass < 4; ++pass) wv[pass] *= ratio;
+    }
+    float psum = 0.f;
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+        const float pv = fast_exp2(lg[pass] - m_new);
+        psum += pv;
+        const int t = pass * 4 + k;
+        if (s < 4) pbuf[t * kG + head] = pv * wv[pass];
+    }
+    st.l = st.l * alpha + psum;
+    if (lane < 4) pbuf[16 * kG + head] = alpha_acc;
+    __syncwarp();
+
+    page_values<kG>(pg, tier, pbuf, lane, alpha_acc, st);
     __syncwarp();
 }
 
+// ---------------------------------------------- two query tokens per pass --
+// Several decode query tokens per sequence (speculative or chunked decode):
+// a launch takes a pair of them, i.e. 8 query heads per kv head, so one page
+// stream serves both and the tensor-core tile's 8 columns are all used.  The
+// shared memory of the query-folded table holds, instead, the pair's query
+// rows (4 arrays of (q[2j], q[2j+1]) for heads 2a, 2a+1, at byte 1024 a +
+// (144 s ^ 16 i) for leaf j = 8s + i) and the warps' weight buffers; every
+// tier's leaves read (cos, sin) from the T1 leaf table, whose grid holds the
+// others (T2 code c is T1 code 16c, T3 code c is T1 code 32c).
+constexpr int kGQ2 = 2 * kG;                          // heads per unit
+constexpr int kMqQOff = kFoldOff;                      // 4 KB of query rows
+constexpr int kMqPbufFloats = 16 * kGQ2 + 2 * kGQ2;    // weights; alpha; valid counts
+constexpr int kMqPbufOff = kMqQOff + 4 * 1024;
+static_assert(kMqPbufOff + kWarps * kMqPbufFloats * 4 <= kFoldOff + kFoldBytes, "pair buffers");
+static_assert((2 * kWarps * kGQ2 + kWarps * kGQ2 * kD) * 4 <= kWarps * kStages * kStageBytes, "pair merge scratch");
+
+// Offsets of one subtree block's 8 leaf codes (into the T1 leaf table) and 8
+// upper codes (into the tier's upper table).
+template <int T>
+__device__ __forceinline__ void block_offsets_mq(const uint8_t* codes, int blk, uint32_t base_rep,
+                                                 const uint32_t (&fl)[8], uint32_t (&lo)[8], uint32_t (&uo)[8])
+{
+    block_offsets<T>(codes, blk, base_rep, fl, lo, uo);
+    if (T == 2) {
+        const uint32_t w = *(const uint32_t*)(codes + blk * 8);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) lo[j] = (((w >> (4 * j)) & 15u) << 12) | base_rep;
+    } else if (T == 3) {
+        const uint32_t lf = *(const uint16_t*)(codes + kP * 32 + blk * 2) | ((uint32_t)codes[kP * 48 + blk] << 16);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) lo[j] = (((lf >> (3 * j)) & 7u) << 13) | base_rep;
+    }
+}
+
+// One subtree block for the 8 heads of a query pair, top down from its
+// weight v: per head, (q[2j], q[2j+1]) . (w cos phi, w sin phi) summed in
+// f32x2 (even, odd) pairs.
+template <int T>
+__device__ __forceinline__ void subtree_mq(float v, const uint32_t (&lo)[8], const uint32_t (&uo)[8],
+                                           const uint8_t* smem, const uint8_t* lut_up, const uint32_t (&fl)[8],
+                                           float2 (&acc2)[kGQ2], bool first)
+{
+    float w2[2], w1[4], wl[8];
+    {
+        const float2 f = *(const float2*)(lut_up + uo[6]);
+        w2[0] = v * f.x;
+        w2[1] = v * f.y;
+    }
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+        const float2 f = *(const float2*)(lut_up + uo[4 + n]);
+        w1[2 * n] = w2[n] * f.x;
+        w1[2 * n + 1] = w2[n] * f.y;
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const float2 f = *(const float2*)(lut_up + uo[m]);
+        wl[2 * m] = w1[m] * f.x;
+        wl[2 * m + 1] = w1[m] * f.y;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float2 f = *(const float2*)(smem + kLutT1 + lo[j]);
+        const float2 kk = make_float2(wl[j] * f.x, wl[j] * f.y);
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const float4 qv = *(const float4*)(smem + kMqQOff + 1024 * a + fl[j]);   // heads 2a, 2a+1
+            const float2 qa = make_float2(qv.x, qv.y), qb = make_float2(qv.z, qv.w);
+            acc2[2 * a] = (first && j == 0) ? __fmul2_rn(qa, kk) : __ffma2_rn(qa, kk, acc2[2 * a]);
+            acc2[2 * a + 1] = (first && j == 0) ? __fmul2_rn(qb, kk) : __ffma2_rn(qb, kk, acc2[2 * a + 1]);
+        }
+    }
+}
+
+// Logits of the 16 tokens of one page for the 8 heads of a query pair, into
+// pbuf[t * 8 + head]; the lane mapping is page_logits' (4 lanes per token,
+// blocks 2q, 2q+1), and the butterfly leaves lane q with heads 2q, 2q+1.
+template <int T>
+__device__ __forceinline__ void page_logits_mq(const uint8_t* pg, const uint8_t* smem, float* pbuf, int lane,
+                                               const uint32_t (&flA)[8])
+{
+    const unsigned full = 0xffffffffu;
+    const int q = lane & 3, k8 = lane >> 2;
+    const bool a_right = k8 & 1;
+    const int sA = 2 * q + (k8 & 1), sB = sA ^ 1;
+    constexpr int kBase = T == 1 ? kLutT1 : T == 2 ? kLutT2 : kLutT3;
+    constexpr int kUp = T == 1 ? 128 : 0;
+    const uint8_t* lut_up = smem + kBase + kUp;
+    const uint32_t rep = (uint32_t)(lane & 15) << 3;
+    const uint8_t* codes = pg + Tier<1>::f.off_codes;
+    uint32_t flB[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) flB[i] = flA[i] ^ 144u;
+    const uint32_t side6 = (uint32_t)(q >> 1) << 2, side5 = (uint32_t)(q & 1) << 2;
+    const int base = lane & ~3;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        const int t = pass * 8 + k8;
+        uint32_t lo[8], uo[8];
+        block_offsets_mq<T>(codes, t * 8 + sA, rep, flA, lo, uo);
+        const uint32_t topB = block_top<T>(codes, t * 8 + sB, rep);
+        const uint32_t top2 = (a_right ? topB : uo[7]) | ((a_right ? uo[7] : topB) << 16);
+        const uint32_t w4 = __shfl_sync(full, top2, base + (q >> 1));
+        const uint32_t w5 = __shfl_sync(full, top2, base + 2);
+        const uint32_t w6 = __shfl_sync(full, top2, base + 3);
+        const uint32_t o4 = (w4 >> (16 * (q & 1))) & 0xffffu;
+        const uint32_t o5 = (w5 >> (16 * (q >> 1))) & 0xffffu;
+        const uint32_t o6 = w6 & 0xffffu;
+        float v = __half2float(((const __half*)pg)[t]) * kLogitScale;
+        v *= *(const float*)(lut_up + o6 + side6);
+        v *= *(const float*)(lut_up + o5 + side5);
+        const float2 f4 = *(const float2*)(lut_up + o4);
+        const float vA = v * (a_right ? f4.y : f4.x), vB = v * (a_right ? f4.x : f4.y);
+        float2 acc2[kGQ2];
+        subtree_mq<T>(vA, lo, uo, smem, lut_up, flA, acc2, true);
+        block_offsets_mq<T>(codes, t * 8 + sB, rep, flB, lo, uo);
+        subtree_mq<T>(vB, lo, uo, smem, lut_up, flB, acc2, false);
+        float acc[kGQ2];
+#pragma unroll
+        for (int h = 0; h < kGQ2; ++h) acc[h] = acc2[h].x + acc2[h].y;
+        // sum over the token's 4 lanes: xor 2 keeps heads 4 b1 .., xor 1 keeps
+        // heads 4 b1 + 2 b0 .. = 2q, 2q+1
+        const bool b1 = q >> 1, b0 = q & 1;
+        float x[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+            x[h] = (b1 ? acc[4 + h] : acc[h]) + __shfl_xor_sync(full, b1 ? acc[h] : acc[4 + h], 2);
+        float y[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) y[h] = (b0 ? x[2 + h] : x[h]) + __shfl_xor_sync(full, b0 ? x[h] : x[2 + h], 1);
+        *(float2*)(pbuf + t * kGQ2 + 2 * q) = make_float2(y[0], y[1]);
+    }
+}
+
+// One staged page for a query pair.  valid0 / valid1: tokens of the page the
+// pair's first / second query sees (the second sees one more token; 0 when
+// the launch has one query).  A head that has seen no token yet keeps an
+// empty state (max -inf, sum 0).
+__device__ __forceinline__ void process_page_mq(const uint8_t* pg, int tier, int valid0, int valid1, const uint8_t* smem,
+                                                float* pbuf, int lane, const uint32_t (&fl)[8], WarpState& st)
+{
+    const unsigned full = 0xffffffffu;
+    const int k = lane >> 3, hh = lane & 7;   // softmax: head hh, tokens 4 pass + k
+    if (lane == 0) {
+        ((int*)pbuf)[16 * kGQ2 + kGQ2] = valid0;
+        ((int*)pbuf)[16 * kGQ2 + kGQ2 + 1] = valid1;
+    }
+    if (tier == 1) page_logits_mq<1>(pg, smem, pbuf, lane, fl);
+    else if (tier == 2) page_logits_mq<2>(pg, smem, pbuf, lane, fl);
+    else page_logits_mq<3>(pg, smem, pbuf, lane, fl);
+    __syncwarp();
+    const int valid = ((const int*)pbuf)[16 * kGQ2 + kGQ2 + (hh >> 2)];
+    const int vmax = max(((const int*)pbuf)[16 * kGQ2 + kGQ2], ((const int*)pbuf)[16 * kGQ2 + kGQ2 + 1]);
+    float lg[4];
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass)
+        lg[pass] = pass * 4 + k < valid ? pbuf[(pass * 4 + k) * kGQ2 + hh] : -INFINITY;
+    __syncwarp();
+    float pm = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
+    pm = fmaxf(pm, __shfl_xor_sync(full, pm, 8));
+    pm = fmaxf(pm, __shfl_xor_sync(full, pm, 16));
+    const float m_new = fmaxf(st.m, pm);
+    const float alpha = m_new == -INFINITY ? 1.f : fast_exp2(st.m - m_new);
+    st.m = m_new;
+    const __half* vs = (const __half*)(pg + 2 * kP);
+    float wv[4];
+    bool big = false;
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+        const int t = pass * 4 + k;
+        wv[pass] = t < vmax ? __half2float(vs[t]) * st.sc : 0.f;
+        big |= wv[pass] > kWeightMax;
+    }
+    float alpha_acc = alpha;
+    if (__any_sync(full, big)) {
+        float vm = fmaxf(fmaxf(wv[0], wv[1]), fmaxf(wv[2], wv[3]));
+        vm = fmaxf(vm, __shfl_xor_sync(full, vm, 8));
+        vm = fmaxf(vm, __shfl_xor_sync(full, vm, 16));
+        const float ratio = pow2_floor(kWeightMax / vm);
+        st.sc *= ratio;
+        alpha_acc *= ratio;
+#pragma unroll
+        for (int pass = 0; pass < 4; ++pass) wv[pass] *= ratio;
+    }
+    float psum = 0.f;
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+        const float pv = lg[pass] == -INFINITY ? 0.f : fast_exp2(lg[pass] - m_new);
+        psum += pv;
+        pbuf[(pass * 4 + k) * kGQ2 + hh] = pv * wv[pass];
+    }
+    st.l = st.l * alpha + psum;
+    if (lane < kGQ2) pbuf[16 * kGQ2 + hh] = alpha_acc;
+    __syncwarp();
+    page_values<kGQ2>(pg, tier, pbuf, lane, alpha_acc, st);
+    __syncwarp();
+}
+
+// Output row of head hh (0 .. heads per unit - 1) of unit (b, g): query
+// token q0 + hh / 4, query head 4g + hh % 4.
+__device__ __forceinline__ int64_t out_row(const DecodeParams& p, int b, int g, int hh)
+{
+    return ((int64_t)b * p.nq + p.q0 + (hh >> 2)) * p.H_q + g * kG + (hh & 3);
+}
+
 // ------------------------------------------------------------ decode --
+// NQ = 1: one query token (4 heads per unit); NQ = 2: a pair (8 heads).
+template <int NQ>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
 {
+    constexpr int GQ = NQ == 1 ? kG : kGQ2;   // heads per unit
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const unsigned full = 0xffffffffu;
@@ -675,7 +901,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
 #pragma unroll
     for (int i = 0; i < 8; ++i) fl[i] = (144u * (uint32_t)(2 * (lane & 3) + ((lane >> 2) & 1))) ^ (16u * i);
     uint8_t* stage = smem + kStageOff + w * kStages * kStageBytes;
-    float* pbuf = (float*)(smem + kPbufOff) + w * kPbufFloats;
+    float* pbuf = NQ == 1 ? (float*)(smem + kPbufOff) + w * kPbufFloats
+                          : (float*)(smem + kMqPbufOff) + w * kMqPbufFloats;
     const uint32_t bar0 = smem_u32(smem + kBarOff + w * kStages * 8);
     if (lane == 0) {
         mbar_init(bar0, 1);
@@ -691,8 +918,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
     bool failed = false;
 
     float* ms_m = (float*)(smem + kStageOff);   // merge scratch, aliases the ring
-    float* ms_l = ms_m + kWarps * kG;
-    float* ms_o = ms_l + kWarps * kG;
+    float* ms_l = ms_m + kWarps * GQ;
+    float* ms_o = ms_l + kWarps * GQ;
 
     for (int32_t x = lo; x < hi;) {
         const int u = find_unit(p.unit_start, p.n_units, x);
@@ -701,7 +928,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
         const int b = u / p.H_kv, g = u % p.H_kv;
         const int32_t pa = x - us, pe = seg_end - us;   // unit-local page range
         const int64_t first = p.page_offsets[b];
-        const int len = p.seq_lens[b];
+        // tokens seen by the (first) query of this launch, and by the second
+        const int len = p.seq_lens[b] - (p.nq - 1 - p.q0);
+        const int len2 = p.npair == 2 ? len + 1 : 0;
         const int32_t* ptab = p.page_table + (int64_t)g * p.total_pages + first;
 
         // Split [pa, pe) among the warps by weight.  Warp w first sums slice w
@@ -718,25 +947,41 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
             sum = __reduce_add_sync(full, sum);
             if (lane == 0) wsum[w] = sum;
         }
-        // query-folded leaf table for this unit (the previous segment ended
-        // with a barrier, so no warp still reads the old one)
-        for (int e = tid; e < 16 * kLeaves; e += kThreads) {
-            const int code = e >> 6, j = e & 63;
-            const float2 cs = *(const float2*)(smem + kLeafT2 + code * 8);
-            float v[kG];
-#pragma unroll
-            for (int h = 0; h < kG; ++h) {
-                const float* qh = p.q + ((int64_t)b * p.H_q + g * kG + h) * kD;
-                v[h] = fmaf(qh[2 * j + 1], cs.y, qh[2 * j] * cs.x);
+        if constexpr (NQ == 1) {
+            // query-folded leaf table for this unit (the previous segment ended
+            // with a barrier, so no warp still reads the old one)
+            for (int e = tid; e < 16 * kLeaves; e += kThreads) {
+                const int code = e >> 6, j = e & 63;
+                const float2 cs = *(const float2*)(smem + kLeafT2 + code * 8);
+                float v[kG];
+    #pragma unroll
+                for (int h = 0; h < kG; ++h) {
+                    const float* qh = p.q + out_row(p, b, g, h) * kD;
+                    v[h] = fmaf(qh[2 * j + 1], cs.y, qh[2 * j] * cs.x);
+                }
+                const uint32_t off = ((uint32_t)code << 10) + 128u * (j >> 3) + 16u * ((j & 7) ^ (j >> 3));
+                *(float4*)(smem + kFoldOff + off) = make_float4(v[0], v[1], v[2], v[3]);
             }
-            const uint32_t off = ((uint32_t)code << 10) + 128u * (j >> 3) + 16u * ((j & 7) ^ (j >> 3));
-            *(float4*)(smem + kFoldOff + off) = make_float4(v[0], v[1], v[2], v[3]);
-        }
-        for (int e = tid; e < 2 * kLeaves; e += kThreads) {   // q for T1 leaves
-            const int half = e >= kLeaves, j = e & 63, sj = j >> 3, ij = j & 7;
-            const float* q0 = p.q + ((int64_t)b * p.H_q + g * kG + 2 * half) * kD + 2 * j;
-            const float* q1 = q0 + kD;
-            *(float4*)(smem + kQOff + 1024 * half + ((144 * sj) ^ (16 * ij))) = make_float4(q0[0], q0[1], q1[0], q1[1]);
+            for (int e = tid; e < 2 * kLeaves; e += kThreads) {   // q for T1 leaves
+                const int half = e >= kLeaves, j = e & 63, sj = j >> 3, ij = j & 7;
+                const float* q0 = p.q + out_row(p, b, g, 2 * half) * kD + 2 * j;
+                const float* q1 = q0 + kD;
+                *(float4*)(smem + kQOff + 1024 * half + ((144 * sj) ^ (16 * ij))) = make_float4(q0[0], q0[1], q1[0], q1[1]);
+            }
+        } else {   // the pair's query rows (the previous segment ended with a barrier)
+            for (int e = tid; e < 4 * kLeaves; e += kThreads) {
+                const int a = e >> 6, j = e & 63, sj = j >> 3, ij = j & 7;
+                float v[4];
+#pragma unroll
+                for (int hp = 0; hp < 2; ++hp) {
+                    const int hh = 2 * a + hp;
+                    const bool live = (hh >> 2) < p.npair;
+                    const float* qh = p.q + out_row(p, b, g, live ? hh : 0) * kD + 2 * j;
+                    v[2 * hp] = live ? qh[0] : 0.f;
+                    v[2 * hp + 1] = live ? qh[1] : 0.f;
+                }
+                *(float4*)(smem + kMqQOff + 1024 * a + ((144 * sj) ^ (16 * ij))) = make_float4(v[0], v[1], v[2], v[3]);
+            }
         }
         __syncthreads();
         int32_t ra, rb;   // this warp's unit-local page range
@@ -848,9 +1093,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
                 break;
             }
             const uint8_t* pg = stage + cur * kStageBytes;
-            const int valid = min(kP, len - lp_cur * kP);
             const int t = entry_tier(e_cur);
-            process_page(pg, t, valid, smem, pbuf, lane, fl, st);
+            if constexpr (NQ == 1) {
+                const int valid = min(kP, len - lp_cur * kP);
+                process_page(pg, t, valid, smem, pbuf, lane, fl, st);
+            } else {
+                const int v0 = max(0, min(kP, len - lp_cur * kP)), v1 = max(0, min(kP, len2 - lp_cur * kP));
+                process_page_mq(pg, t, v0, v1, smem, pbuf, lane, fl, st);
+            }
             cur ^= 1;
             lp_cur = lp_nxt;
             e_cur = e_nxt;
@@ -864,45 +1114,49 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
         __syncthreads();   // every warp is done with its ring
         {
             const int s = lane & 7;
-            const int head = (s & 1) * 2 + ((s >> 1) & 1);
-            if (lane < 4) {
-                ms_m[w * kG + head] = st.m;
-                ms_l[w * kG + head] = lt;
+            // the softmax head of lane (k, s): (s & 1) * 2 + ((s >> 1) & 1) for
+            // one query (lanes s, s + 4 alike), s for a pair
+            const int head = NQ == 1 ? (s & 1) * 2 + ((s >> 1) & 1) : s;
+            if (lane < GQ) {
+                ms_m[w * GQ + head] = st.m;
+                ms_l[w * GQ + head] = lt;
             }
             // accumulator (tile m, i): dim 16m + g + 8*(i >> 1), head 2c + (i & 1)
             const int gq = lane >> 2, cq = lane & 3;
             const float inv_sc = 1.0f / st.sc;   // exact: sc is a power of two
-            if (cq < 2) {
+            if (2 * cq < GQ) {
 #pragma unroll
                 for (int m = 0; m < 8; ++m)
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        ms_o[(w * kG + 2 * cq + (i & 1)) * kD + 16 * m + gq + 8 * (i >> 1)] = st.acc[m][i] * inv_sc;
+                        ms_o[(w * GQ + 2 * cq + (i & 1)) * kD + 16 * m + gq + 8 * (i >> 1)] = st.acc[m][i] * inv_sc;
             }
         }
         __syncthreads();
-        for (int idx = tid; idx < kG * kD; idx += kThreads) {
+        for (int idx = tid; idx < GQ * kD; idx += kThreads) {
             const int h = idx >> 7, dim = idx & (kD - 1);
             float M = -INFINITY;
 #pragma unroll
-            for (int ww = 0; ww < kWarps; ++ww) M = fmaxf(M, ms_m[ww * kG + h]);
+            for (int ww = 0; ww < kWarps; ++ww) M = fmaxf(M, ms_m[ww * GQ + h]);
             float L = 0.f, O = 0.f;
             if (M != -INFINITY) {
 #pragma unroll
                 for (int ww = 0; ww < kWarps; ++ww) {
-                    const float mw = ms_m[ww * kG + h];
+                    const float mw = ms_m[ww * GQ + h];
                     if (mw == -INFINITY) continue;
                     const float sc = exp2f(mw - M);
-                    L += ms_l[ww * kG + h] * sc;
-                    O += ms_o[(ww * kG + h) * kD + dim] * sc;
+                    L += ms_l[ww * GQ + h] * sc;
+                    O += ms_o[(ww * GQ + h) * kD + dim] * sc;
                 }
             }
             if (pa == 0 && seg_end == ue) {   // the whole unit: final result
-                const int64_t row = (int64_t)b * p.H_q + g * kG + h;
-                p.out[row * kD + dim] = L > 0.f ? O / L : 0.f;
-                if (dim == 0) p.lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+                if ((h >> 2) < p.npair) {
+                    const int64_t row = out_row(p, b, g, h);
+                    p.out[row * kD + dim] = L > 0.f ? O / L : 0.f;
+                    if (dim == 0) p.lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+                }
             } else {
-                float* part = p.partial + ((int64_t)(blockIdx.x + u) * kG + h) * kPartStride;
+                float* part = p.partial + ((int64_t)(blockIdx.x + u) * GQ + h) * kPartStride;
                 part[4 + dim] = O;
                 if (dim == 0) {
                     part[0] = M;
@@ -917,15 +1171,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
 }
 
 // --------------------------------------------------------------- merge --
-__global__ void __launch_bounds__(kG * kD) merge_kernel(DecodeParams p)
+template <int GQ>
+__global__ void __launch_bounds__(GQ * kD) merge_kernel(DecodeParams p)
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");   // decode_kernel's partials are visible
     const int u = blockIdx.x;
     const int h = threadIdx.x >> 7, dim = threadIdx.x & (kD - 1);
+    if ((h >> 2) >= p.npair) return;   // no such query in this launch
     const int32_t P = p.unit_start[p.n_units];
     const int32_t us = p.unit_start[u], ue = p.unit_start[u + 1];
     const int b = u / p.H_kv, g = u % p.H_kv;
-    const int64_t row = (int64_t)b * p.H_q + g * kG + h;
+    const int64_t row = out_row(p, b, g, h);
     if (ue == us) {   // no pages: nothing attended
         p.out[row * kD + dim] = 0.f;
         if (dim == 0) p.lse[row] = -INFINITY;
@@ -942,12 +1198,12 @@ __global__ void __launch_bounds__(kG * kD) merge_kernel(DecodeParams p)
     float M = -INFINITY;
     for (int c = c0; c <= c1; ++c)
         if (cta_bound(c, P, p.n_cta) < cta_bound(c + 1, P, p.n_cta))
-            M = fmaxf(M, p.partial[((int64_t)(c + u) * kG + h) * kPartStride]);
+            M = fmaxf(M, p.partial[((int64_t)(c + u) * GQ + h) * kPartStride]);
     float L = 0.f, O = 0.f;
     if (M != -INFINITY) {
         for (int c = c0; c <= c1; ++c) {
             if (cta_bound(c, P, p.n_cta) == cta_bound(c + 1, P, p.n_cta)) continue;
-            const float* part = p.partial + ((int64_t)(c + u) * kG + h) * kPartStride;
+            const float* part = p.partial + ((int64_t)(c + u) * GQ + h) * kPartStride;
             if (part[0] == -INFINITY) continue;
             const float sc = exp2f(part[0] - M);
             L += part[1] * sc;
@@ -962,8 +1218,10 @@ __global__ void __launch_bounds__(kG * kD) merge_kernel(DecodeParams p)
 // programmatic dependents (PDL): each may start its prologue while the kernel
 // before it finishes, and waits (griddepcontrol.wait) before reading that
 // kernel's results.
+template <int NQ>
 void launch_decode(const DecodeParams& p, cudaStream_t s)
 {
+    constexpr int GQ = NQ == 1 ? kG : kGQ2;
     plan_kernel<<<1, 1024, 0, s>>>(p);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -975,11 +1233,11 @@ void launch_decode(const DecodeParams& p, cudaStream_t s)
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, decode_kernel, p);
+    cudaLaunchKernelEx(&cfg, decode_kernel<NQ>, p);
     cfg.gridDim = dim3(p.n_units);
-    cfg.blockDim = dim3(kG * kD);
+    cfg.blockDim = dim3(GQ * kD);
     cfg.dynamicSmemBytes = 0;
-    cudaLaunchKernelEx(&cfg, merge_kernel, p);
+    cudaLaunchKernelEx(&cfg, merge_kernel<GQ>, p);
 }
 
 int sm_count(int n_sm)
@@ -1000,12 +1258,100 @@ int pick_ctas(int H_kv, int64_t total_pages, int n_sm)
     return (int)n;
 }
 
-size_t ws_layout(int B, int H_kv, int n_cta, size_t* part_off)
+// Workspace: unit_start [n_units + 1] | partials [n_cta + n_units][GQ][kPartStride].
+size_t ws_layout(int B, int H_kv, int n_cta, int GQ, size_t* part_off)
 {
     size_t n_units = (size_t)B * H_kv;
     size_t off = ((n_units + 1) * 4 + 255) / 256 * 256;
     *part_off = off;
-    return off + (size_t)(n_cta + n_units) * kG * kPartStride * 4;
+    return off + (size_t)(n_cta + n_units) * GQ * kPartStride * 4;
+}
+
+// Argument checks shared by the decode entry points; fills everything in p
+// but the query-token fields and the workspace pointers.
+sphkv_status fill_params(const char* fn, const sphkv_cache* c, int32_t H_q, const float* q, float* out, float* lse,
+                         int32_t* status_dev, DecodeParams& p)
+{
+    if (!c || !q || !out || !lse) {
+        sphkv_set_error("%s: null argument", fn);
+        return SPHKV_ERR_ARG;
+    }
+    if (c->B <= 0 || c->H_kv <= 0 || !c->page_offsets || !c->seq_lens || !c->page_table ||
+        c->total_pages < 0) {
+        sphkv_set_error("%s: bad cache descriptor", fn);
+        return SPHKV_ERR_ARG;
+    }
+    if (H_q != kG * c->H_kv) {
+        sphkv_set_error("%s: H_q / H_kv must be %d (got H_q=%d, H_kv=%d)", fn, kG, H_q, c->H_kv);
+        return SPHKV_ERR_ARG;
+    }
+    if ((uintptr_t)q & 15) {
+        sphkv_set_error("%s: q must be 16-byte aligned", fn);
+        return SPHKV_ERR_ARG;
+    }
+    if ((int64_t)c->H_kv * c->total_pages > 0x7fffffffLL || (int64_t)c->B * c->H_kv > (1 << 24)) {
+        sphkv_set_error("%s: cache too large for 32-bit page indices", fn);
+        return SPHKV_ERR_ARG;
+    }
+    p = DecodeParams{};
+    for (int t = 1; t <= 3; ++t) {
+        p.pool[t] = c->pool[t - 1];
+        p.pool_pages[t] = c->pool[t - 1] ? c->pool_pages[t - 1] : 0;
+        if ((uintptr_t)c->pool[t - 1] & 15) {
+            sphkv_set_error("%s: pool %d is not 16-byte aligned", fn, t);
+            return SPHKV_ERR_ARG;
+        }
+    }
+    p.n_cta = pick_ctas(c->H_kv, c->total_pages, sm_count(0));
+    p.page_offsets = c->page_offsets;
+    p.seq_lens = c->seq_lens;
+    p.page_table = c->page_table;
+    p.total_pages = c->total_pages;
+    p.B = c->B;
+    p.H_kv = c->H_kv;
+    p.H_q = H_q;
+    p.n_units = c->B * c->H_kv;
+    p.q = q;
+    p.out = out;
+    p.lse = lse;
+    p.status = status_dev;
+    p.nq = 1;
+    p.q0 = 0;
+    p.npair = 1;
+    p.len_shift = 0;
+    return SPHKV_OK;
+}
+
+// Opt the decode kernels into their shared memory, once per device and thread.
+sphkv_status ensure_smem(const char* fn)
+{
+    static thread_local int attr_dev = -1;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        sphkv_set_error("%s: no usable current device", fn);
+        return SPHKV_ERR_DEVICE;
+    }
+    if (attr_dev != dev) {
+        if (cudaFuncSetAttribute(decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+                cudaSuccess) {
+            sphkv_set_error("%s: cannot reserve %d bytes of shared memory", fn, kSmemBytes);
+            return SPHKV_ERR_DEVICE;
+        }
+        attr_dev = dev;
+    }
+    return SPHKV_OK;
+}
+
+sphkv_status launched(const char* fn)
+{
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) {
+        sphkv_set_error("%s: launch failed: %s", fn, cudaGetErrorString(err));
+        return SPHKV_ERR_DEVICE;
+    }
+    return SPHKV_OK;
 }
 
 }  // namespace
@@ -1019,84 +1365,78 @@ extern "C" size_t sphkv_decode_workspace_bytes(int32_t B, int32_t H_q, int32_t H
     (void)H_q;
     if (B <= 0 || H_kv <= 0 || total_pages < 0) return 0;
     size_t off;
-    return ws_layout(B, H_kv, pick_ctas(H_kv, total_pages, sm_count(n_sm)), &off);
+    return ws_layout(B, H_kv, pick_ctas(H_kv, total_pages, sm_count(n_sm)), kG, &off);
 }
 
 extern "C" sphkv_status sphkv_decode_attention(const sphkv_cache* c, int32_t H_q, const float* q,
                                                float* out, float* lse, void* workspace,
                                                size_t ws_bytes, int32_t* status_dev, void* stream)
 {
-    if (!c || !q || !out || !lse || !workspace) {
-        sphkv_set_error("sphkv_decode_attention: null argument");
+    const char* fn = "sphkv_decode_attention";
+    DecodeParams p;
+    sphkv_status st = fill_params(fn, c, H_q, q, out, lse, status_dev, p);
+    if (st != SPHKV_OK) return st;
+    if (!workspace || ((uintptr_t)workspace & 255)) {
+        sphkv_set_error("%s: workspace must be non-null and 256-byte aligned", fn);
         return SPHKV_ERR_ARG;
     }
-    if (c->B <= 0 || c->H_kv <= 0 || !c->page_offsets || !c->seq_lens || !c->page_table ||
-        c->total_pages < 0) {
-        sphkv_set_error("sphkv_decode_attention: bad cache descriptor");
-        return SPHKV_ERR_ARG;
-    }
-    if (H_q != kG * c->H_kv) {
-        sphkv_set_error("sphkv_decode_attention: H_q / H_kv must be %d (got H_q=%d, H_kv=%d)", kG, H_q,
-                        c->H_kv);
-        return SPHKV_ERR_ARG;
-    }
-    if (((uintptr_t)q & 15) || ((uintptr_t)workspace & 255)) {
-        sphkv_set_error("sphkv_decode_attention: q must be 16-byte and workspace 256-byte aligned");
-        return SPHKV_ERR_ARG;
-    }
-    if ((int64_t)c->H_kv * c->total_pages > 0x7fffffffLL || (int64_t)c->B * c->H_kv > (1 << 24)) {
-        sphkv_set_error("sphkv_decode_attention: cache too large for 32-bit page indices");
-        return SPHKV_ERR_ARG;
-    }
-    DecodeParams p{};
-    for (int t = 1; t <= 3; ++t) {
-        p.pool[t] = c->pool[t - 1];
-        p.pool_pages[t] = c->pool[t - 1] ? c->pool_pages[t - 1] : 0;
-        if ((uintptr_t)c->pool[t - 1] & 15) {
-            sphkv_set_error("sphkv_decode_attention: pool %d is not 16-byte aligned", t);
-            return SPHKV_ERR_ARG;
-        }
-    }
-    const int n_sm = sm_count(0);
-    p.n_cta = pick_ctas(c->H_kv, c->total_pages, n_sm);
     size_t part_off;
-    const size_t need = ws_layout(c->B, c->H_kv, p.n_cta, &part_off);
+    const size_t need = ws_layout(c->B, c->H_kv, p.n_cta, kG, &part_off);
     if (ws_bytes < need) {
-        sphkv_set_error("sphkv_decode_attention: workspace %zu bytes < %zu needed", ws_bytes, need);
+        sphkv_set_error("%s: workspace %zu bytes < %zu needed", fn, ws_bytes, need);
         return SPHKV_ERR_ARG;
     }
-    p.page_offsets = c->page_offsets;
-    p.seq_lens = c->seq_lens;
-    p.page_table = c->page_table;
-    p.total_pages = c->total_pages;
-    p.B = c->B;
-    p.H_kv = c->H_kv;
-    p.H_q = H_q;
-    p.n_units = c->B * c->H_kv;
-    p.q = q;
-    p.out = out;
-    p.lse = lse;
     p.unit_start = (int32_t*)workspace;
     p.partial = (float*)((uint8_t*)workspace + part_off);
-    p.status = status_dev;
+    if ((st = ensure_smem(fn)) != SPHKV_OK) return st;
+    launch_decode<1>(p, (cudaStream_t)stream);
+    return launched(fn);
+}
 
-    static thread_local int attr_dev = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (attr_dev != dev) {
-        if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kSmemBytes) != cudaSuccess) {
-            sphkv_set_error("sphkv_decode_attention: cannot reserve %d bytes of shared memory", kSmemBytes);
-            return SPHKV_ERR_DEVICE;
-        }
-        attr_dev = dev;
+extern "C" size_t sphkv_decode_mq_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int64_t total_pages,
+                                                  int32_t n_sm)
+{
+    (void)H_q;
+    if (B <= 0 || H_kv <= 0 || total_pages < 0) return 0;
+    size_t off;
+    return ws_layout(B, H_kv, pick_ctas(H_kv, total_pages, sm_count(n_sm)), kGQ2, &off);
+}
+
+extern "C" sphkv_status sphkv_decode_attention_mq(const sphkv_cache* c, int32_t n_q, int32_t H_q, const float* q,
+                                                  float* out, float* lse, void* workspace, size_t ws_bytes,
+                                                  int32_t* status_dev, void* stream)
+{
+    const char* fn = "sphkv_decode_attention_mq";
+    DecodeParams p;
+    sphkv_status st = fill_params(fn, c, H_q, q, out, lse, status_dev, p);
+    if (st != SPHKV_OK) return st;
+    if (n_q < 1 || n_q > 1024) {
+        sphkv_set_error("%s: n_q must be in 1..1024 (got %d)", fn, n_q);
+        return SPHKV_ERR_ARG;
     }
-    cudaStream_t s = (cudaStream_t)stream;
-    launch_decode(p, s);
-    cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess) {
-        sphkv_set_error("sphkv_decode_attention: launch failed: %s", cudaGetErrorString(err));
-        return SPHKV_ERR_DEVICE;
+    if (!workspace || ((uintptr_t)workspace & 255)) {
+        sphkv_set_error("%s: workspace must be non-null and 256-byte aligned", fn);
+        return SPHKV_ERR_ARG;
+    }
+    size_t part_off;
+    const size_t need = ws_layout(c->B, c->H_kv, p.n_cta, kGQ2, &part_off);
+    if (ws_bytes < need) {
+        sphkv_set_error("%s: workspace %zu bytes < %zu needed", fn, ws_bytes, need);
+        return SPHKV_ERR_ARG;
+    }
+    p.unit_start = (int32_t*)workspace;
+    p.partial = (float*)((uint8_t*)workspace + part_off);
+    if ((st = ensure_smem(fn)) != SPHKV_OK) return st;
+    p.nq = n_q;
+    // query tokens two at a time; the launches share the workspace in stream
+    // order (each plan waits for the previous merge)
+    for (int q0 = 0; q0 < n_q; q0 += 2) {
+        p.q0 = q0;
+        p.npair = min(2, n_q - q0);
+        p.len_shift = n_q - q0 - p.npair;
+        if (p.npair == 2) launch_decode<2>(p, (cudaStream_t)stream);
+        else launch_decode<1>(p, (cudaStream_t)stream);
+        if ((st = launched(fn)) != SPHKV_OK) return st;
     }
     return SPHKV_OK;
 }
@@ -1121,50 +1461,21 @@ extern "C" sphkv_status sphkv_decode_attention_noalloc(const sphkv_cache* c, int
                                                        float* out, float* lse, int32_t* status_dev,
                                                        void* stream)
 {
-    if (!c || !q || !out || !lse) {
-        sphkv_set_error("sphkv_decode_attention_noalloc: null argument");
-        return SPHKV_ERR_ARG;
-    }
-    if (c->B <= 0 || c->H_kv <= 0 || !c->page_offsets || !c->seq_lens || !c->page_table ||
-        c->total_pages < 0) {
-        sphkv_set_error("sphkv_decode_attention_noalloc: bad cache descriptor");
-        return SPHKV_ERR_ARG;
-    }
-    if (H_q != kG * c->H_kv) {
-        sphkv_set_error("sphkv_decode_attention_noalloc: H_q / H_kv must be %d (got H_q=%d, H_kv=%d)", kG,
-                        H_q, c->H_kv);
-        return SPHKV_ERR_ARG;
-    }
-    if ((uintptr_t)q & 15) {
-        sphkv_set_error("sphkv_decode_attention_noalloc: q must be 16-byte aligned");
-        return SPHKV_ERR_ARG;
-    }
-    if ((int64_t)c->H_kv * c->total_pages > 0x7fffffffLL || (int64_t)c->B * c->H_kv > (1 << 24)) {
-        sphkv_set_error("sphkv_decode_attention_noalloc: cache too large for 32-bit page indices");
-        return SPHKV_ERR_ARG;
-    }
-    DecodeParams p{};
-    for (int t = 1; t <= 3; ++t) {
-        p.pool[t] = c->pool[t - 1];
-        p.pool_pages[t] = c->pool[t - 1] ? c->pool_pages[t - 1] : 0;
-        if ((uintptr_t)c->pool[t - 1] & 15) {
-            sphkv_set_error("sphkv_decode_attention_noalloc: pool %d is not 16-byte aligned", t);
-            return SPHKV_ERR_ARG;
-        }
-    }
-    p.n_cta = pick_ctas(c->H_kv, c->total_pages, sm_count(0));
+    const char* fn = "sphkv_decode_attention_noalloc";
+    DecodeParams p;
+    sphkv_status st = fill_params(fn, c, H_q, q, out, lse, status_dev, p);
+    if (st != SPHKV_OK) return st;
     size_t part_off;
-    const size_t need = ws_layout(c->B, c->H_kv, p.n_cta, &part_off);
+    const size_t need = ws_layout(c->B, c->H_kv, p.n_cta, kG, &part_off);
     if (need > kNoAllocScratchBytes) {
-        sphkv_set_error(
-            "sphkv_decode_attention_noalloc: this cache needs %zu bytes of scratch but the static area holds "
-            "%zu; use sphkv_decode_attention with a caller workspace",
-            need, kNoAllocScratchBytes);
+        sphkv_set_error("%s: this cache needs %zu bytes of scratch but the static area holds %zu; use "
+                        "sphkv_decode_attention with a caller workspace",
+                        fn, need, kNoAllocScratchBytes);
         return SPHKV_ERR_ARG;
     }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-        sphkv_set_error("sphkv_decode_attention_noalloc: no usable current device");
+        sphkv_set_error("%s: no usable current device", fn);
         return SPHKV_ERR_DEVICE;
     }
     void* scratch = nullptr;
@@ -1177,40 +1488,17 @@ extern "C" sphkv_status sphkv_decode_attention_noalloc(const sphkv_cache* c, int
             void* a = nullptr;
             const cudaError_t e = cudaGetSymbolAddress(&a, g_noalloc_scratch);
             if (e != cudaSuccess || !a) {
-                sphkv_set_error("sphkv_decode_attention_noalloc: cudaGetSymbolAddress failed: %s",
-                                cudaGetErrorString(e));
+                sphkv_set_error("%s: cudaGetSymbolAddress failed: %s", fn, cudaGetErrorString(e));
                 return SPHKV_ERR_DEVICE;
             }
-            if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-                cudaSuccess) {
-                sphkv_set_error("sphkv_decode_attention_noalloc: cannot reserve %d bytes of shared memory",
-                                kSmemBytes);
-                return SPHKV_ERR_DEVICE;
-            }
+            if ((st = ensure_smem(fn)) != SPHKV_OK) return st;
             g_noalloc_addr[dev] = a;
         }
         scratch = g_noalloc_addr[dev];
     }
-    p.page_offsets = c->page_offsets;
-    p.seq_lens = c->seq_lens;
-    p.page_table = c->page_table;
-    p.total_pages = c->total_pages;
-    p.B = c->B;
-    p.H_kv = c->H_kv;
-    p.H_q = H_q;
-    p.n_units = c->B * c->H_kv;
-    p.q = q;
-    p.out = out;
-    p.lse = lse;
+    if ((st = ensure_smem(fn)) != SPHKV_OK) return st;
     p.unit_start = (int32_t*)scratch;
     p.partial = (float*)((uint8_t*)scratch + part_off);
-    p.status = status_dev;
-    cudaStream_t s = (cudaStream_t)stream;
-    launch_decode(p, s);
-    const cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess) {
-        sphkv_set_error("sphkv_decode_attention_noalloc: launch failed: %s", cudaGetErrorString(err));
-        return SPHKV_ERR_DEVICE;
-    }
-    return SPHKV_OK;
+    launch_decode<1>(p, (cudaStream_t)stream);
+    return launched(fn);
 }

@@ -225,6 +225,32 @@ sphkv_status sphkv_decode_attention(const sphkv_cache* cache, int32_t H_q, const
 sphkv_status sphkv_decode_attention_noalloc(const sphkv_cache* cache, int32_t H_q, const float* q,
                                             float* out, float* lse, int32_t* status_dev, void* stream);
 
+/*
+ * sphkv_decode_mq_workspace_bytes / sphkv_decode_attention_mq -- ADA decode
+ *   for n_q query tokens per sequence at once (speculative or chunked decode).
+ *   Spherical KV, Abstract (the decode path is meant to fuse with the
+ *   surrounding decode work); the multi-token form is this library's reading:
+ *   query token i (0 <= i < n_q) of sequence b is causal, it sees the first
+ *   seq_len[b] - (n_q - 1 - i) tokens (the last query token sees them all;
+ *   the cache already holds the tokens the earlier queries precede), and
+ *   otherwise attends exactly as in sphkv_decode_attention.
+ *   q: [B][n_q][H_q][128] fp32, out: [B][n_q][H_q][128] fp32, lse:
+ *   [B][n_q][H_q] fp32.  A query that sees no kept token gets out = 0,
+ *   lse = -inf.  Query tokens are taken two at a time: one pass over the pages
+ *   serves both (8 query heads per kv head on the tensor-core tile); an odd
+ *   last token runs alone.  Pages are therefore read ceil(n_q / 2) times.
+ *   1 <= n_q <= 1024, H_q / H_kv must be 4.  workspace: device, 256-byte
+ *   aligned, at least sphkv_decode_mq_workspace_bytes(B, H_q, H_kv,
+ *   total_pages, n_sm) bytes (n_sm = 0: the current device's SM count); the
+ *   launches of one call reuse it in stream order.  Errors as
+ *   sphkv_decode_attention, plus SPHKV_ERR_ARG for n_q out of range.
+ */
+size_t sphkv_decode_mq_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int64_t total_pages,
+                                       int32_t n_sm);
+sphkv_status sphkv_decode_attention_mq(const sphkv_cache* cache, int32_t n_q, int32_t H_q, const float* q,
+                                       float* out, float* lse, void* workspace, size_t ws_bytes,
+                                       int32_t* status_dev, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -227,6 +227,24 @@ def cache_attention(cache, q, units):
     return out, lse
 
 
+def multi_query_attention(cache, q, units, n_q):
+    """Decode attention for n_q query tokens per sequence, q [B, n_q, H_q, 128].
+    Reading (the pages describe one decode query per step; several query
+    tokens per step, as in speculative or chunked decode, are this project's
+    extension): query token i is causal and sees the first
+    seq_len - (n_q - 1 - i) tokens, so the last one sees them all.  Each token
+    is then plain single-query attention (cache_attention) over its prefix.
+    Returns out [n_q, n, G, 128], lse [n_q, n, G]."""
+    q = np.asarray(q)
+    outs, lses = [], []
+    for i in range(n_q):
+        lens = np.maximum(np.asarray(cache["seq_lens"], np.int64) - (n_q - 1 - i), 0).astype(np.int32)
+        o, l = cache_attention(dict(cache, seq_lens=lens), q[:, i], units)
+        outs.append(o)
+        lses.append(l)
+    return np.stack(outs), np.stack(lses)
+
+
 def rdr_assign(page_offsets, seq_lens, utility, eps, budget, n_sink, n_recent, H_kv,
                tiers_init=None):
     """Lagrangian tier assignment.  utility: [H_kv, total_pages*16] f32.

@@ -25,7 +25,7 @@ def test_library_exports_every_declared_symbol():
     build.build()
     lib = ctypes.CDLL(_lib.LIB_PATH)
     names = _declared()
-    assert len(names) == 9, names
+    assert len(names) == 11, names
     missing = [n for n in names if not hasattr(lib, n)]
     assert not missing, missing
     # the binding covers the same names
@@ -44,6 +44,8 @@ def test_host_helpers_agree_with_the_format():
     assert L.sphkv_decode_workspace_bytes(8, 32, 8, 8 * 2048, 148) > 0
     assert L.sphkv_rdr_workspace_bytes(16, 8, 16 * 2064) >= 8 * 16 * 2064 * 9
     assert L.sphkv_decode_workspace_bytes(0, 32, 8, 10, 148) == 0
+    assert L.sphkv_decode_mq_workspace_bytes(8, 32, 8, 8 * 2048, 148) > \
+        L.sphkv_decode_workspace_bytes(8, 32, 8, 8 * 2048, 148)
 
 
 def test_workloads_are_deterministic_and_shaped():

@@ -185,6 +185,50 @@ def test_all_dropped_and_q_zero():
     assert np.all(np.abs(lse[1] - np.log(kept)) <= 1e-4)
 
 
+@pytest.mark.parametrize("n_q", [1, 2, 3, 4])
+def test_multi_query_decode(n_q):
+    """n_q causal query tokens per sequence (query i sees the first
+    seq_len - (n_q - 1 - i) tokens), through sphkv_decode_attention_mq, against
+    the oracle: ragged lengths, drops, a one-token sequence and an empty one."""
+    torch = _torch()
+    w = W.make("ragged64", seq_lens=[700, 33, 1, 0, 2049], H_kv=2, H_q=8)
+    w.permute_pools = True
+    cache = gpu_cache(w)
+    rng = np.random.default_rng(17 + n_q)
+    q = rng.standard_normal((w.B, n_q, w.H_q, 128)).astype(np.float32)
+    out, lse = cache.decode_mq(to_torch(q, torch.float32))
+    cache.check()
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    ref = oracle_full_cache(w)
+    units = [(b, g) for b in range(w.B) for g in range(w.H_kv)]
+    ro, rl = oracle.multi_query_attention(ref, q, units, n_q)
+    for i in range(n_q):
+        for k, (b, g) in enumerate(units):
+            assert_close(out[b, i, 4 * g:4 * g + 4], lse[b, i, 4 * g:4 * g + 4], ro[i, k], rl[i, k],
+                         f"query {i} unit {(b, g)}")
+    if n_q == 1:   # the same kernel as sphkv_decode_attention
+        o1, l1 = _decode(cache, q[:, 0])
+        assert np.array_equal(o1, out[:, 0]) and np.array_equal(l1, lse[:, 0])
+
+
+def test_multi_query_full_size_sampled():
+    """Two query tokens per sequence at the 32k workload's full size, on the
+    launch path bench.py --n-q 2 times; sampled units against the oracle."""
+    torch = _torch()
+    w = W.make("llama32k")
+    cache = gpu_cache(w)
+    rng = np.random.default_rng(23)
+    q = rng.standard_normal((w.B, 2, w.H_q, 128)).astype(np.float32)
+    out, lse = cache.decode_mq(to_torch(q, torch.float32))
+    cache.check()
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    for b, g in [(0, 0), (5, 7)]:
+        for i in range(2):
+            lens = np.maximum(w.seq_lens - (1 - i), 0)
+            ro, rl = oracle_unit(w, b, g, q[:, i], lens=lens)
+            assert_close(out[b, i, 4 * g:4 * g + 4], lse[b, i, 4 * g:4 * g + 4], ro, rl, f"query {i} unit {(b, g)}")
+
+
 def test_physical_permutation_is_bit_identical():
     torch = _torch()
     w = W.make("ragged64", seq_lens=[3000, 1111, 2222], H_kv=2, H_q=8)

@@ -281,6 +281,38 @@ def test_dropped_pages_contribute_exactly_zero():
     assert np.array_equal(lse[0], lse2)
 
 
+def test_multi_query_is_causal_prefix_attention():
+    """Pin (multi-token decode): query token i of n_q equals, bit for bit,
+    attention over the kept tokens among the first seq_len - (n_q - 1 - i),
+    each decoded on its own; n_q = 1 is plain single-query attention."""
+    rng = np.random.default_rng(9)
+    tiers = [1, 2, 0, 3, 1, 2, 3, 1]
+    seq_len = 8 * 16 - 5
+    cache, K, V = _small_cache(rng, tiers, seq_len)
+    n_q = 3
+    q = rng.standard_normal((1, n_q, 4, 128))
+    out, lse = oracle.multi_query_attention(cache, q, [(0, 0)], n_q)
+    o1, l1 = oracle.cache_attention(cache, q[:, n_q - 1], [(0, 0)])
+    assert np.array_equal(out[n_q - 1], o1) and np.array_equal(lse[n_q - 1], l1)
+    for i in range(n_q):
+        n_i = seq_len - (n_q - 1 - i)
+        keep_k, keep_v = [], []
+        for t in range(n_i):
+            tier = tiers[t // 16]
+            if tier == 0:
+                continue
+            c = oracle.encode(K[t:t + 1, 0], V[t:t + 1, 0], tier)
+            bl, bu, _ = TIERS[tier]
+            keep_k.append(oracle.decode_keys(c["leaf"], c["up"], c["r16"], bl, bu)[0])
+            keep_v.append(oracle.decode_values(c["vq"], c["s16"])[0])
+        o2, l2 = oracle.attention(np.array(keep_k), np.array(keep_v), q[0, i])
+        assert np.array_equal(out[i, 0], o2) and np.array_equal(lse[i, 0], l2), i
+    # a sequence shorter than n_q: the early query tokens see nothing
+    short = dict(cache, seq_lens=np.array([1], np.int32))
+    o, l = oracle.multi_query_attention(short, q, [(0, 0)], n_q)
+    assert np.all(np.isneginf(l[:n_q - 1])) and np.all(o[:n_q - 1] == 0) and np.all(np.isfinite(l[n_q - 1]))
+
+
 def test_special_cases():
     """Pin: q = 0 gives the mean of the kept values and lse = ln(#kept); one
     kept token gives its value and its logit; no kept token gives out = 0,
