@@ -40,6 +40,9 @@
 //             p * vscale * sc are split into f16 hi + lo parts (two MMAs),
 //             keeping ~22 bits.
 //   merge  -- one CTA per unit whose pages were split over several CTAs.
+// decode_kernel<1> serves one query token per sequence (4 query heads per kv
+// head); decode_kernel<2> serves a pair of causal query tokens (8 heads), see
+// "two query tokens per pass" below.
 #include <mutex>
 
 #include "common.cuh"
