@@ -1114,7 +1114,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
         float lt = st.l;   // lanes s and s+4 duplicate: sum over k only
         lt += __shfl_xor_sync(full, lt, 8);
         lt += __shfl_xor_sync(full, lt, 16);
-        __syncthreads();   // every warp is done with its ring
+        // every warp is done with its ring; a timed-out copy in any warp ends
+        // the whole CTA after this segment (every warp leaves the loop together)
+        failed = __syncthreads_or(failed);
         {
             const int s = lane & 7;
             // the softmax head of lane (k, s): (s & 1) * 2 + ((s >> 1) & 1) for
