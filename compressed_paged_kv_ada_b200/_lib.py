@@ -52,37 +52,42 @@ def lib() -> ctypes.CDLL:
     """Load libsphkv.so (built in-tree by compressed_paged_kv_ada_b200.build)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError(f"{LIB_PATH} is missing: run `python -m compressed_paged_kv_ada_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
-        c, P = ctypes, ctypes.c_void_p
-        L.sphkv_page_bytes.restype = c.c_int
-        L.sphkv_page_bytes.argtypes = [c.c_int]
-        L.sphkv_last_error.restype = c.c_char_p
-        L.sphkv_last_error.argtypes = []
-        L.sphkv_encode.restype = c.c_int
-        L.sphkv_encode.argtypes = [c.POINTER(sphkv_cache), P, P, c.c_int, P, P, c.c_int64, P, P]
-        L.sphkv_rdr_workspace_bytes.restype = c.c_size_t
-        L.sphkv_rdr_workspace_bytes.argtypes = [c.c_int32, c.c_int32, c.c_int64]
-        L.sphkv_rdr_assign.restype = c.c_int
-        L.sphkv_rdr_assign.argtypes = [c.POINTER(sphkv_cache), P, c.POINTER(c.c_double), c.c_int64,
-                                       c.c_int32, c.c_int32, P, P, P, P, c.c_size_t, P, P]
-        L.sphkv_build_page_table.restype = c.c_int
-        L.sphkv_build_page_table.argtypes = [P, c.c_int64, P, P, P, P, P, P, P]
-        L.sphkv_decode_workspace_bytes.restype = c.c_size_t
-        L.sphkv_decode_workspace_bytes.argtypes = [c.c_int32, c.c_int32, c.c_int32, c.c_int64, c.c_int32]
-        L.sphkv_decode_attention.restype = c.c_int
-        L.sphkv_decode_attention.argtypes = [c.POINTER(sphkv_cache), c.c_int32, P, P, P, P, c.c_size_t,
-                                             P, P]
-        L.sphkv_decode_attention_noalloc.restype = c.c_int
-        L.sphkv_decode_attention_noalloc.argtypes = [c.POINTER(sphkv_cache), c.c_int32, P, P, P, P, P]
-        L.sphkv_decode_mq_workspace_bytes.restype = c.c_size_t
-        L.sphkv_decode_mq_workspace_bytes.argtypes = [c.c_int32, c.c_int32, c.c_int32, c.c_int64, c.c_int32]
-        L.sphkv_decode_attention_mq.restype = c.c_int
-        L.sphkv_decode_attention_mq.argtypes = [c.POINTER(sphkv_cache), c.c_int32, c.c_int32, P, P, P, P,
-                                                c.c_size_t, P, P]
-        _lib = L
+        _lib = load(LIB_PATH)
     return _lib
+
+
+def load(path: str) -> ctypes.CDLL:
+    """Open a build of the library at `path` with the C signatures declared."""
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: run `python -m compressed_paged_kv_ada_b200.build`")
+    L = ctypes.CDLL(path)
+    c, P = ctypes, ctypes.c_void_p
+    L.sphkv_page_bytes.restype = c.c_int
+    L.sphkv_page_bytes.argtypes = [c.c_int]
+    L.sphkv_last_error.restype = c.c_char_p
+    L.sphkv_last_error.argtypes = []
+    L.sphkv_encode.restype = c.c_int
+    L.sphkv_encode.argtypes = [c.POINTER(sphkv_cache), P, P, c.c_int, P, P, c.c_int64, P, P]
+    L.sphkv_rdr_workspace_bytes.restype = c.c_size_t
+    L.sphkv_rdr_workspace_bytes.argtypes = [c.c_int32, c.c_int32, c.c_int64]
+    L.sphkv_rdr_assign.restype = c.c_int
+    L.sphkv_rdr_assign.argtypes = [c.POINTER(sphkv_cache), P, c.POINTER(c.c_double), c.c_int64,
+                                   c.c_int32, c.c_int32, P, P, P, P, c.c_size_t, P, P]
+    L.sphkv_build_page_table.restype = c.c_int
+    L.sphkv_build_page_table.argtypes = [P, c.c_int64, P, P, P, P, P, P, P]
+    L.sphkv_decode_workspace_bytes.restype = c.c_size_t
+    L.sphkv_decode_workspace_bytes.argtypes = [c.c_int32, c.c_int32, c.c_int32, c.c_int64, c.c_int32]
+    L.sphkv_decode_attention.restype = c.c_int
+    L.sphkv_decode_attention.argtypes = [c.POINTER(sphkv_cache), c.c_int32, P, P, P, P, c.c_size_t,
+                                         P, P]
+    L.sphkv_decode_attention_noalloc.restype = c.c_int
+    L.sphkv_decode_attention_noalloc.argtypes = [c.POINTER(sphkv_cache), c.c_int32, P, P, P, P, P]
+    L.sphkv_decode_mq_workspace_bytes.restype = c.c_size_t
+    L.sphkv_decode_mq_workspace_bytes.argtypes = [c.c_int32, c.c_int32, c.c_int32, c.c_int64, c.c_int32]
+    L.sphkv_decode_attention_mq.restype = c.c_int
+    L.sphkv_decode_attention_mq.argtypes = [c.POINTER(sphkv_cache), c.c_int32, c.c_int32, P, P, P, P,
+                                            c.c_size_t, P, P]
+    return L
 
 
 def _check(fn: str, code: int):

@@ -2,6 +2,11 @@
 
     python -m compressed_paged_kv_ada_b200.build [--force] [--verbose]
 
+It also builds libsphkv_testhooks.so, the same library with decode.cu
+compiled with -DSPHKV_TEST_HOOKS, which only the tests load (they use it to
+make a bounded device wait run out without any fault).  The product library
+is built without the flag.
+
 encode.cu and rdr.cu are compiled with -fmad=false: their fp64 arithmetic must
 not be contracted into fused multiply-adds (codes and tier decisions are
 compared bit for bit with a plain fp64 reference).
@@ -17,6 +22,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsphkv.so")
+TEST_LIB = os.path.join(HERE, "libsphkv_testhooks.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -36,23 +42,30 @@ def _deps():
     return files
 
 
+def _link(objs, out):
+    tmp = out + ".tmp"
+    subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart"])
+    os.replace(tmp, out)
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     newest = max(os.path.getmtime(f) for f in _deps())
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:
+    if (not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest and os.path.exists(TEST_LIB)
+            and os.path.getmtime(TEST_LIB) >= newest):
         return LIB
-    objs = []
-    for src, extra in SOURCES.items():
-        obj = os.path.join(BUILD, src.replace(".cu", ".o"))
-        cmd = [NVCC, *ARCH, *COMMON, *extra, "-c", os.path.join(CSRC, src), "-o", obj]
+    objs = {}
+    for src, extra in list(SOURCES.items()) + [("decode.cu#hooks", ["-DSPHKV_TEST_HOOKS"])]:
+        name = src.split("#")[0]
+        obj = os.path.join(BUILD, src.replace(".cu", "").replace("#", "_") + ".o")
+        cmd = [NVCC, *ARCH, *COMMON, *extra, "-c", os.path.join(CSRC, name), "-o", obj]
         if verbose:
             cmd += ["-Xptxas", "-v"]
             print(" ".join(cmd), flush=True)
         subprocess.check_call(cmd)
-        objs.append(obj)
-    tmp = LIB + ".tmp"
-    subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart"])
-    os.replace(tmp, LIB)
+        objs[src] = obj
+    _link([objs[s] for s in SOURCES], LIB)
+    _link([objs[s] for s in SOURCES if s != "decode.cu"] + [objs["decode.cu#hooks"]], TEST_LIB)
     return LIB
 
 

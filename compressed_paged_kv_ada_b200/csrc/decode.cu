@@ -43,6 +43,7 @@
 // decode_kernel<1> serves one query token per sequence (4 query heads per kv
 // head); decode_kernel<2> serves a pair of causal query tokens (8 heads), see
 // "two query tokens per pass" below.
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -120,6 +121,12 @@ struct DecodeParams {
     // lse: [B][nq][H_q].  len_shift = nq - q0 - npair: the launch's page range
     // is that of its last query token.
     int nq, q0, npair, len_shift;
+#ifdef SPHKV_TEST_HOOKS
+    // Test builds only (environment SPHKV_TEST_SKIP_FIRST_COPY): warp 0 of
+    // CTA 0 skips its first page copy, so its bounded wait runs out (after a
+    // short limit) and the call reports SPHKV_ERR_TIMEOUT without any fault.
+    int test_skip_copy;
+#endif
     const float* q;
     float* out;
     float* lse;
@@ -177,9 +184,10 @@ __device__ inline bool mbar_try_wait(uint32_t bar, uint32_t parity)
 }
 
 // Bounded wait on an mbarrier phase; false if the limit ran out.
+template <long Limit = kWaitLimit>
 __device__ inline bool mbar_wait(uint32_t bar, uint32_t parity)
 {
-    for (long i = 0; i < kWaitLimit; ++i) {
+    for (long i = 0; i < Limit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if (i > 16) __nanosleep(64);
     }
@@ -1080,11 +1088,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
         int32_t lp_cur = 0, e_cur = 0, lp_nxt = 0, e_nxt = 0;
         bool have_cur = advance(cur_c, lp_cur, e_cur);
         int cur = 0;
-        if (have_cur) issue(0, e_cur);
+#ifdef SPHKV_TEST_HOOKS
+        const bool skip_first = p.test_skip_copy && blockIdx.x == 0 && w == 0 && x == lo;
+#else
+        constexpr bool skip_first = false;
+#endif
+        if (have_cur && !skip_first) issue(0, e_cur);
         while (have_cur) {
             const bool have_nxt = advance(cur_c, lp_nxt, e_nxt);
             if (have_nxt) issue(cur ^ 1, e_nxt);
+#ifdef SPHKV_TEST_HOOKS
+            const bool ok = p.test_skip_copy ? mbar_wait<(1L << 12)>(bar0 + 8 * cur, (phase >> cur) & 1)
+                                             : mbar_wait(bar0 + 8 * cur, (phase >> cur) & 1);
+#else
             const bool ok = mbar_wait(bar0 + 8 * cur, (phase >> cur) & 1);
+#endif
             phase ^= 1u << cur;
             if (!ok) {
                 if (lane == 0) report(p.status, SPHKV_ERR_TIMEOUT);
@@ -1324,6 +1342,10 @@ sphkv_status fill_params(const char* fn, const sphkv_cache* c, int32_t H_q, cons
     p.q0 = 0;
     p.npair = 1;
     p.len_shift = 0;
+#ifdef SPHKV_TEST_HOOKS
+    const char* skip = std::getenv("SPHKV_TEST_SKIP_FIRST_COPY");
+    p.test_skip_copy = skip && skip[0] && skip[0] != '0';
+#endif
     return SPHKV_OK;
 }
 
