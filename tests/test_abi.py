@@ -31,6 +31,9 @@ def test_library_exports_every_declared_symbol():
     # the binding covers the same names
     for n in names:
         assert n in _lib._EXPORTS or n in ("sphkv_last_error",), n
+    # the test-hook build (loaded only by tests) exports the same interface
+    T = ctypes.CDLL(build.TEST_LIB)
+    assert not [n for n in names if not hasattr(T, n)]
 
 
 def test_host_helpers_agree_with_the_format():
