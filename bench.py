@@ -98,6 +98,14 @@ def profiled_traffic(kernel_src: str, summary: str):
         return None
 
 
+def served_units(w, n_q: int = 1) -> int:
+    """Token-heads one step serves: query token i of n_q attends to the first
+    seq_len - (n_q - 1 - i) tokens (all of them for a single query), for every
+    query head; dropped tokens count as served work."""
+    lens = np.asarray(w.seq_lens, np.int64)
+    return int(sum(np.maximum(lens - (n_q - 1 - i), 0).sum() for i in range(n_q))) * w.H_q
+
+
 def algorithmic_bytes(w) -> int:
     """Exact bytes the decode must move for one step: the bits of every kept
     token, one page-table entry per token-holding page, q, out and lse."""
@@ -337,8 +345,7 @@ def run_gpu(args):
     ms_total = start.elapsed_time(end)
     call_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
     ms_step = ms_total / args.steps
-    # token-heads served: query token i attends to seq_len - (n_q - 1 - i) tokens
-    units = int(sum(np.maximum(w.seq_lens - (n_q - 1 - i), 0).sum() for i in range(n_q))) * w.H_q
+    units = served_units(w, n_q)
     t_all = [ms_step]
     u_all = [units]
     if world > 1:

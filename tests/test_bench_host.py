@@ -79,3 +79,13 @@ def test_profiled_traffic_goes_stale(tmp_path):
     assert bench.profiled_traffic(str(src), str(summ)) == 1234
     src.write_text("kernel v2")
     assert bench.profiled_traffic(str(src), str(summ)) is None
+
+
+def test_served_units_count_each_query_tokens_prefix():
+    """One query: all tokens of every sequence for every query head; n_q
+    causal tokens: token i serves seq_len - (n_q - 1 - i), never below 0."""
+    w = W.make("ragged64", seq_lens=[5, 1, 0, 40], H_kv=2, H_q=8)
+    assert bench.served_units(w) == (5 + 1 + 0 + 40) * 8
+    # n_q = 3: token 0 sees len - 2, token 1 len - 1, token 2 len
+    per_seq = [max(5 - 2, 0) + 4 + 5, 0 + 0 + 1, 0, 38 + 39 + 40]
+    assert bench.served_units(w, 3) == sum(per_seq) * 8
