@@ -23,6 +23,7 @@ def test_page_wait_timeout_reports_and_context_recovers(monkeypatch):
 
     from compressed_paged_kv_ada_b200 import _lib, build
 
+    build.build()   # no-op when both libraries are current
     T = _lib.load(build.TEST_LIB)
     w = W.make("ragged64", seq_lens=[2049, 1500], H_kv=2, H_q=8)
     cache = gpu_cache(w)
