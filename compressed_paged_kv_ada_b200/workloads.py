@@ -139,16 +139,19 @@ class Workload:
         """q [B, H_q, 128] fp32 ~ N(0, 1); step > 0 gives later decode steps."""
         return _rng(self.seed, self.cfg, "q", step).standard_normal((self.B, self.H_q, D), dtype=np.float32)
 
-    def utility(self) -> np.ndarray:
+    def utility(self, lens: Optional[np.ndarray] = None) -> np.ndarray:
         """Per token and kv head utility [H_kv, total_pages*16] f32:
         LogNormal(0, 1) / (1 + age/4096), age = len - 1 - position; slots
-        without a token are 0."""
+        without a token are 0.  The LogNormal draw of a slot does not depend
+        on len (one draw per reserved slot), so utilities stay consistent as
+        a sequence grows; only the age term changes."""
+        lens = self.seq_lens if lens is None else np.asarray(lens)
         out = np.zeros((self.H_kv, self.total_pages * PAGE), np.float32)
         po = self.page_offsets
         for b in range(self.B):
-            n = int(self.seq_lens[b])
+            n = int(lens[b])
             r = _rng(self.seed, self.cfg, "util", b)
-            u = r.lognormal(0.0, 1.0, size=(self.H_kv, n))
+            u = r.lognormal(0.0, 1.0, size=(self.H_kv, int(self.cap_pages[b]) * PAGE))[:, :n]
             age = (n - 1 - np.arange(n)).astype(np.float64)
             out[:, po[b] * PAGE: po[b] * PAGE + n] = (u / (1.0 + age / 4096.0)).astype(np.float32)
         return out

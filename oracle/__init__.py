@@ -76,6 +76,17 @@ def lib():
         L.orc_rdr_assign.restype = c.c_int
         L.orc_rdr_assign.argtypes = [c.c_int, c.c_int, c.c_int64, P, P, P, P, c.c_int64,
                                      c.c_int, c.c_int, P, P, P]
+        L.orc_rdr_rerun.restype = c.c_int
+        L.orc_rdr_rerun.argtypes = [c.c_int, c.c_int, c.c_int64, P, P, P, P, c.c_int64,
+                                    c.c_int, c.c_int, P, P, P]
+        L.orc_transcode_token.restype = None
+        L.orc_transcode_token.argtypes = [c.c_int, c.c_int, P, P, c.c_uint16, P, P, P, P, P]
+        L.orc_migrate.restype = c.c_int
+        L.orc_migrate.argtypes = [c.c_int, c.c_int, c.c_int64, P, P, P, P, P, P, P, P, P, P, P, P]
+        L.orc_set_keep.restype = c.c_int
+        L.orc_set_keep.argtypes = [c.c_int, c.c_int, c.c_int64, P, P, P, P, P, P, P, P]
+        L.orc_merge_partials.restype = None
+        L.orc_merge_partials.argtypes = [c.c_int, c.c_int64, c.c_int, P, P, P, P]
         L.orc_num_threads.restype = c.c_int
         L.orc_num_threads.argtypes = []
         _lib = L
@@ -169,6 +180,45 @@ def attention(khat, vhat, q):
     out = np.zeros((n_q, d), np.float64)
     lse = np.zeros(n_q, np.float64)
     lib().orc_attention(n, d, _p(khat), _p(vhat), n_q, _p(q), _p(out), _p(lse))
+    return out, lse
+
+
+def set_keep(cache, keep):
+    """Per-token keep/drop: keep [H_kv, total_pages * 16] (nonzero = keep), in
+    RDR's utility layout.  Sets (drop) or clears (keep) the drop flag, the sign
+    bit of the stored radius, of every present token of every kept page of the
+    cache dict's pools, in place.  Dropped tokens are then skipped by
+    cache_attention exactly as if deleted."""
+    po = _c(cache["page_offsets"], np.int32)
+    sl = _c(cache["seq_lens"], np.int32)
+    pt = _c(cache["page_table"], np.int32)
+    H_kv, total_pages = pt.shape
+    keep = _c(keep, np.uint8)
+    assert keep.shape == (H_kv, total_pages * PAGE)
+    pools = cache["pools"]
+    flat = []
+    for t, p in enumerate(pools):
+        assert p.flags["C_CONTIGUOUS"] and p.dtype == np.uint8
+        flat.append(p if p.size else np.zeros((1, page_bytes(t + 1)), np.uint8))
+    pool_pages = np.array([p.shape[0] if p.size else 0 for p in pools], np.int64)
+    st = lib().orc_set_keep(sl.size, H_kv, total_pages, _p(po), _p(sl), _p(pt), _p(flat[0]), _p(flat[1]),
+                            _p(flat[2]), _p(pool_pages), _p(keep))
+    if st != 0:
+        raise ValueError(f"oracle set_keep status {st}")
+
+
+def merge_partials(out_parts, lse_parts):
+    """Log-sum-exp combine of attention results over disjoint key sets:
+    out_parts [n_parts, ..., d], lse_parts [n_parts, ...].  Returns (out, lse)
+    of attention over the union of the parts' keys."""
+    op = _c(out_parts, np.float64)
+    lp = _c(lse_parts, np.float64)
+    n_parts = op.shape[0]
+    d = op.shape[-1]
+    n_rows = int(np.prod(lp.shape[1:], dtype=np.int64))
+    out = np.zeros(op.shape[1:], np.float64)
+    lse = np.zeros(lp.shape[1:], np.float64)
+    lib().orc_merge_partials(n_parts, n_rows, d, _p(op), _p(lp), _p(out), _p(lse))
     return out, lse
 
 
@@ -267,6 +317,61 @@ def rdr_assign(page_offsets, seq_lens, utility, eps, budget, n_sink, n_recent, H
     if st != 0:
         raise ValueError(f"oracle rdr status {st}")
     return tiers, float(lam[0]), int(nbytes[0])
+
+
+def rdr_rerun(page_offsets, seq_lens, utility, eps, budget, n_sink, n_recent, tiers):
+    """RDR again on a cache that already holds codes: each page may only keep
+    its tier or become coarser (drop included); forced pages keep the finest
+    tier allowed.  tiers: the current [H_kv, total_pages] tiers.  Returns
+    (new tiers, lambda, bytes) or raises OverflowError if infeasible."""
+    po = _c(page_offsets, np.int32)
+    sl = _c(seq_lens, np.int32)
+    util = _c(utility, np.float32)
+    eps = _c(eps, np.float64)
+    t = _c(tiers, np.uint8).copy()
+    H_kv, total_pages = t.shape
+    lam = np.zeros(1, np.float64)
+    nbytes = np.zeros(1, np.int64)
+    st = lib().orc_rdr_rerun(sl.size, H_kv, total_pages, _p(po), _p(sl), _p(util), _p(eps), int(budget),
+                             n_sink, n_recent, _p(t), _p(lam), _p(nbytes))
+    if st == 3:
+        raise OverflowError("forced pages alone exceed the budget")
+    if st != 0:
+        raise ValueError(f"oracle rdr status {st}")
+    return t, float(lam[0]), int(nbytes[0])
+
+
+def transcode_token(t_from, t_to, leaf, up, s16, vq):
+    """One token's codes from tier t_from to the coarser (or same) tier t_to.
+    Returns dict(leaf, up, s16, vq); the radius does not change."""
+    leaf2 = np.zeros(D // 2, np.uint8)
+    up2 = np.zeros(D // 2 - 1, np.uint8)
+    s2 = np.zeros(1, np.uint16)
+    vq2 = np.zeros(D, np.int8)
+    lib().orc_transcode_token(t_from, t_to, _p(_c(leaf, np.uint8)), _p(_c(up, np.uint8)), int(s16),
+                              _p(_c(vq, np.int8)), _p(leaf2), _p(up2), _p(s2), _p(vq2))
+    return dict(leaf=leaf2, up=up2, s16=int(s2[0]), vq=vq2)
+
+
+def migrate(cache, new_table, new_counts):
+    """Rewrite the cache dict's tokens into fresh pools laid out by new_table
+    ([H_kv, total_pages] entries; new_counts pages per tier), transcoding the
+    pages whose tier became coarser.  Returns the new pools."""
+    po = _c(cache["page_offsets"], np.int32)
+    sl = _c(cache["seq_lens"], np.int32)
+    ot = _c(cache["page_table"], np.int32)
+    nt = _c(new_table, np.int32)
+    H_kv, total_pages = ot.shape
+    old = [p if p.size else np.zeros((1, page_bytes(t + 1)), np.uint8) for t, p in enumerate(cache["pools"])]
+    old_pages = np.array([p.shape[0] if p.size else 0 for p in cache["pools"]], np.int64)
+    new = [np.zeros((int(new_counts[t]), page_bytes(t + 1)), np.uint8) for t in range(3)]
+    newp = [p if p.size else np.zeros((1, page_bytes(t + 1)), np.uint8) for t, p in enumerate(new)]
+    new_pages = np.array([int(c) for c in new_counts], np.int64)
+    st = lib().orc_migrate(sl.size, H_kv, total_pages, _p(po), _p(sl), _p(ot), _p(old[0]), _p(old[1]), _p(old[2]),
+                           _p(old_pages), _p(nt), _p(newp[0]), _p(newp[1]), _p(newp[2]), _p(new_pages))
+    if st != 0:
+        raise ValueError(f"oracle migrate status {st}")
+    return [newp[t] if new[t].size else new[t] for t in range(3)]
 
 
 def encode_cache(K, V, tok_seq, tok_pos, page_offsets, page_table, pool_pages):

@@ -323,6 +323,38 @@ void orc_attention(int64_t n_keys, int d, const double* khat, const double* vhat
     free(l);
 }
 
+/* Combine attention results over disjoint key sets of the same query rows
+ * (split-KV: each part attended to its own keys; Spherical KV, Abstract:
+ * long-context inference; the log-sum-exp combine is the one the decode path
+ * uses to merge its own splits).  With M = max_r lse_r and w_r =
+ * e^(lse_r - M):  out = sum_r w_r out_r / sum_r w_r,  lse = M + ln sum_r w_r,
+ * which is attention over the union of the parts' keys.  A part with
+ * lse = -inf (no keys) has w_r = 0; if every part is empty, out = 0 and
+ * lse = -inf.  out_parts [n_parts][n_rows][d], lse_parts [n_parts][n_rows]. */
+void orc_merge_partials(int n_parts, int64_t n_rows, int d, const double* out_parts, const double* lse_parts,
+                        double* out, double* lse)
+{
+    for (int64_t i = 0; i < n_rows; ++i) {
+        double M = -INFINITY;
+        for (int r = 0; r < n_parts; ++r)
+            if (lse_parts[(int64_t)r * n_rows + i] > M) M = lse_parts[(int64_t)r * n_rows + i];
+        double* o = out + i * d;
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        if (M == -INFINITY) { lse[i] = -INFINITY; continue; }
+        double Z = 0.0;
+        for (int r = 0; r < n_parts; ++r) {
+            double l = lse_parts[(int64_t)r * n_rows + i];
+            if (l == -INFINITY) continue;
+            double w = exp(l - M);
+            Z += w;
+            const double* orow = out_parts + ((int64_t)r * n_rows + i) * d;
+            for (int c = 0; c < d; ++c) o[c] += w * orow[c];
+        }
+        for (int c = 0; c < d; ++c) o[c] /= Z;
+        lse[i] = M + log(Z);
+    }
+}
+
 /* -------------------------------------------------------- page format -- */
 
 /* The codes of one token regrouped into 8 subtree blocks, one per 8-leaf
@@ -556,6 +588,7 @@ int orc_cache_attention(int B, int H_q, int H_kv, int64_t total_pages, const int
             }
             const uint8_t* page = pools[tier] + phys * (int64_t)orc_page_bytes(tier);
             orc_unpack_token(tier, (int)(t % ORC_PAGE), page, leaf, up, &r16, &s16, vq);
+            if (r16 & 0x8000u) continue; /* the token's drop flag (see orc_set_keep) */
             decode_key_one(ORC_D, leaf, up, r16, ORC_BLEAF[tier], ORC_BUP[tier], K + n * ORC_D, w);
             orc_decode_values(1, ORC_D, vq, &s16, V + n * ORC_D);
             ++n;
@@ -568,20 +601,147 @@ int orc_cache_attention(int B, int H_q, int H_kv, int64_t total_pages, const int
     return status;
 }
 
+/* Transcoding a stored token to a coarser tier, from its codes alone (the
+ * dense key is gone once a page is written).  Reading (the pages give no
+ * rule): each angle is moved to the nearest point of the coarser grid,
+ * computed exactly on the code integers with ties to even, which is what
+ * re-encoding the decoded angle would give without the rounding noise of
+ * atan2; the radius (and its drop flag) is kept; the values are decoded
+ * (code * scale, exact in fp64) and quantised again with the encoder's rule
+ * for the new width. */
+
+/* Round-half-even of num / den for num >= 0, den > 0. */
+static int64_t div_rne(int64_t num, int64_t den)
+{
+    int64_t q = num / den, r = num % den;
+    if (2 * r > den || (2 * r == den && (q & 1))) ++q;
+    return q;
+}
+
+/* Leaf code on the periodic 2^b_from grid -> nearest point of the 2^b_to grid
+ * (b_to <= b_from): c * 2^b_to / 2^b_from, ties to even, modulo 2^b_to. */
+static int transcode_leaf(int c, int b_from, int b_to)
+{
+    return (int)(div_rne((int64_t)c << b_to, (int64_t)1 << b_from) % ((int64_t)1 << b_to));
+}
+
+/* Upper code on the end-inclusive grid with 2^b_from - 1 steps -> nearest
+ * point of the 2^b_to - 1 step grid: c (2^b_to - 1) / (2^b_from - 1), ties to
+ * even (the denominator is odd, so none occur). */
+static int transcode_upper(int c, int b_from, int b_to)
+{
+    return (int)div_rne((int64_t)c * (((int64_t)1 << b_to) - 1), ((int64_t)1 << b_from) - 1);
+}
+
+/* One token from tier t_from to tier t_to (t_to no finer than t_from). */
+void orc_transcode_token(int t_from, int t_to, const uint8_t* leaf, const uint8_t* up, uint16_t s16,
+                         const int8_t* vq, uint8_t* leaf_out, uint8_t* up_out, uint16_t* s16_out, int8_t* vq_out)
+{
+    for (int j = 0; j < ORC_D / 2; ++j) leaf_out[j] = (uint8_t)transcode_leaf(leaf[j], ORC_BLEAF[t_from], ORC_BLEAF[t_to]);
+    for (int j = 0; j < ORC_D / 2 - 1; ++j) up_out[j] = (uint8_t)transcode_upper(up[j], ORC_BUP[t_from], ORC_BUP[t_to]);
+    double v[ORC_D];
+    orc_decode_values(1, ORC_D, vq, &s16, v);
+    double Q = (ORC_VBITS[t_to] == 8) ? 127.0 : 7.0;
+    double a = 0.0;
+    for (int c = 0; c < ORC_D; ++c) a = fmax(a, fabs(v[c]));
+    *s16_out = orc_f64_to_f16(a / Q);
+    double s = orc_f16_to_f64(*s16_out);
+    for (int c = 0; c < ORC_D; ++c) {
+        double t = (s == 0.0) ? 0.0 : rint(v[c] / s);
+        if (t > Q) t = Q;
+        if (t < -Q) t = -Q;
+        vq_out[c] = (int8_t)t;
+    }
+}
+
+/* Rewrite a cache into new pools after its tiers changed (RDR run again):
+ * every present token of a page kept by the new table is transcoded from its
+ * old page into its new page (a page whose tier did not change moves
+ * unchanged: no re-quantisation); pages the new table
+ * drops are not written.  The new pools must be zeroed by the caller.  A page
+ * the new table makes finer than before, or keeps although it was dropped,
+ * cannot be rebuilt from codes: status 6 (the page is skipped). */
+int orc_migrate(int B, int H_kv, int64_t total_pages, const int32_t* page_offsets, const int32_t* seq_lens,
+                const int32_t* old_table, const uint8_t* old1, const uint8_t* old2, const uint8_t* old3,
+                const int64_t* old_pages, const int32_t* new_table, uint8_t* new1, uint8_t* new2, uint8_t* new3,
+                const int64_t* new_pages)
+{
+    const uint8_t* olds[4] = {NULL, old1, old2, old3};
+    uint8_t* news[4] = {NULL, new1, new2, new3};
+    int status = 0;
+    uint8_t leaf[ORC_D / 2], up[ORC_D / 2 - 1], leaf2[ORC_D / 2], up2[ORC_D / 2 - 1];
+    int8_t vq[ORC_D], vq2[ORC_D];
+    for (int g = 0; g < H_kv; ++g)
+        for (int b = 0; b < B; ++b)
+            for (int64_t t = 0; t < seq_lens[b]; ++t) {
+                int64_t lp = (int64_t)g * total_pages + page_offsets[b] + t / ORC_PAGE;
+                int32_t eo = old_table[lp], en = new_table[lp];
+                int to = (int)(((uint32_t)eo) >> 30), tn = (int)(((uint32_t)en) >> 30);
+                int64_t po = (int64_t)(((uint32_t)eo) & 0x3fffffffu), pn = (int64_t)(((uint32_t)en) & 0x3fffffffu);
+                if (tn == 0) continue;
+                if (to == 0 || tn < to || po >= old_pages[to - 1] || pn >= new_pages[tn - 1]) { status = 6; continue; }
+                uint16_t r16, s16, s16b;
+                int slot = (int)(t % ORC_PAGE);
+                orc_unpack_token(to, slot, olds[to] + po * (int64_t)orc_page_bytes(to), leaf, up, &r16, &s16, vq);
+                if (tn == to) /* same tier: the token moves unchanged */
+                    orc_pack_token(tn, slot, leaf, up, r16, s16, vq, news[tn] + pn * (int64_t)orc_page_bytes(tn));
+                else {
+                    orc_transcode_token(to, tn, leaf, up, s16, vq, leaf2, up2, &s16b, vq2);
+                    orc_pack_token(tn, slot, leaf2, up2, r16, s16b, vq2, news[tn] + pn * (int64_t)orc_page_bytes(tn));
+                }
+            }
+    return status;
+}
+
+/* Per-token keep/drop inside kept pages.  Spherical KV, Abstract: RDR makes
+ * keep/drop decisions per token and head.  Reading: a stored radius is
+ * fp16(|k|) >= +0, so its sign bit is free; it is the token's drop flag (1 =
+ * dropped), and attention skips a dropped token exactly as if it had been
+ * deleted.  keep: [H_kv][total_pages * 16] bytes in the layout of RDR's
+ * utility (slot s of logical page i at i * 16 + s); for every present token
+ * (position < seq_len) of every page that is not dropped, the flag is set
+ * when keep is 0 and cleared otherwise.  Pools are modified in place. */
+int orc_set_keep(int B, int H_kv, int64_t total_pages, const int32_t* page_offsets, const int32_t* seq_lens,
+                 const int32_t* page_table, uint8_t* pool1, uint8_t* pool2, uint8_t* pool3,
+                 const int64_t* pool_pages, const uint8_t* keep)
+{
+    uint8_t* pools[4] = {NULL, pool1, pool2, pool3};
+    int status = 0;
+    for (int g = 0; g < H_kv; ++g)
+        for (int b = 0; b < B; ++b)
+            for (int64_t t = 0; t < seq_lens[b]; ++t) {
+                int64_t lp = page_offsets[b] + t / ORC_PAGE;
+                int32_t e = page_table[(int64_t)g * total_pages + lp];
+                int tier = (int)(((uint32_t)e) >> 30);
+                int64_t phys = (int64_t)(((uint32_t)e) & 0x3fffffffu);
+                if (tier == 0) continue;
+                if (phys >= pool_pages[tier - 1]) { status = 6; continue; }
+                uint8_t* r = pools[tier] + phys * (int64_t)orc_page_bytes(tier) + 2 * (t % ORC_PAGE);
+                uint16_t r16 = (uint16_t)get_le(r, 2);
+                int k = keep[(int64_t)g * total_pages * ORC_PAGE + lp * ORC_PAGE + t % ORC_PAGE] != 0;
+                r16 = k ? (uint16_t)(r16 & 0x7fffu) : (uint16_t)(r16 | 0x8000u);
+                put_le(r, 2, r16);
+            }
+    return status;
+}
+
 /* ---------------------------------------------------------------- RDR -- */
 
 /* Lagrangian tier choice for one unit: argmin over t of U*eps[t] + lambda*R[t],
  * ties to the lower index (higher precision).  Index 0..3 = T1, T2, T3, drop. */
-static int rdr_choice(double U, const double* eps, const double* R, double lambda)
+static int rdr_choice(double U, const double* eps, const double* R, double lambda, int first)
 {
-    int best = 0;
-    double bc = U * eps[0] + lambda * R[0];
-    for (int t = 1; t < 4; ++t) {
+    int best = first;
+    double bc = U * eps[first] + lambda * R[first];
+    for (int t = first + 1; t < 4; ++t) {
         double c = U * eps[t] + lambda * R[t];
         if (c < bc) { bc = c; best = t; }
     }
     return best;
 }
+
+/* Tier (1..3, 0 = drop) -> choice index (0..3 = T1, T2, T3, drop). */
+static int tier_index(int tier) { return tier == 0 ? 3 : tier - 1; }
 
 /* Rate-distortion retention.  Units are (kv head g, sequence b, page p) for
  * p < ceil(seq_len/16).  U = sum of the per-token utilities of the valid
@@ -594,10 +754,44 @@ static int rdr_choice(double U, const double* eps, const double* R, double lambd
  * tiers: [H_kv][total_pages], written 1..3 or 0 (drop) for pages that hold
  * tokens; other entries are left untouched.
  * Returns 0, or 3 when the forced pages alone exceed the budget. */
+static int rdr_run(int B, int H_kv, int64_t total_pages, const int32_t* page_offsets, const int32_t* seq_lens,
+                   const float* utility, const double* eps, int64_t budget, int n_sink, int n_recent,
+                   const uint8_t* cap, uint8_t* tiers, double* lambda_out, int64_t* bytes_out);
+
 int orc_rdr_assign(int B, int H_kv, int64_t total_pages, const int32_t* page_offsets,
                    const int32_t* seq_lens, const float* utility, const double* eps,
                    int64_t budget, int n_sink, int n_recent, uint8_t* tiers,
                    double* lambda_out, int64_t* bytes_out)
+{
+    return rdr_run(B, H_kv, total_pages, page_offsets, seq_lens, utility, eps, budget, n_sink, n_recent, NULL,
+                   tiers, lambda_out, bytes_out);
+}
+
+/* RDR run again on a cache whose pages already hold codes (the context has
+ * grown; Spherical KV, AI Summary: retention allocates precision and storage
+ * dynamically by estimated utility).  Reading: a page's codes can only be
+ * made coarser without the dense key, so every unit's choices are limited to
+ * its current tier and the coarser ones (drop included); forced units (first
+ * n_sink, last n_recent pages) keep the finest tier they are allowed, i.e.
+ * T1 if they are T1 and their current tier otherwise.  tiers holds the
+ * current tiers on entry and the new ones on return (pages that hold tokens;
+ * other entries untouched).  Otherwise exactly orc_rdr_assign. */
+int orc_rdr_rerun(int B, int H_kv, int64_t total_pages, const int32_t* page_offsets, const int32_t* seq_lens,
+                  const float* utility, const double* eps, int64_t budget, int n_sink, int n_recent,
+                  uint8_t* tiers, double* lambda_out, int64_t* bytes_out)
+{
+    int64_t n = (int64_t)H_kv * total_pages;
+    uint8_t* cap = (uint8_t*)malloc((size_t)(n > 0 ? n : 1));
+    memcpy(cap, tiers, (size_t)n);
+    int st = rdr_run(B, H_kv, total_pages, page_offsets, seq_lens, utility, eps, budget, n_sink, n_recent, cap,
+                     tiers, lambda_out, bytes_out);
+    free(cap);
+    return st;
+}
+
+static int rdr_run(int B, int H_kv, int64_t total_pages, const int32_t* page_offsets, const int32_t* seq_lens,
+                   const float* utility, const double* eps, int64_t budget, int n_sink, int n_recent,
+                   const uint8_t* cap, uint8_t* tiers, double* lambda_out, int64_t* bytes_out)
 {
     double R[4];
     for (int t = 0; t < 3; ++t) R[t] = (double)orc_page_bytes(t + 1);
@@ -609,6 +803,7 @@ int orc_rdr_assign(int B, int H_kv, int64_t total_pages, const int32_t* page_off
     double* U = (double*)malloc(sizeof(double) * (size_t)(n_units > 0 ? n_units : 1));
     int64_t* idx = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n_units > 0 ? n_units : 1));
     uint8_t* forced = (uint8_t*)malloc((size_t)(n_units > 0 ? n_units : 1));
+    uint8_t* first = (uint8_t*)malloc((size_t)(n_units > 0 ? n_units : 1)); /* finest allowed choice */
     int64_t u = 0, forced_bytes = 0;
     for (int g = 0; g < H_kv; ++g)
         for (int b = 0; b < B; ++b) {
@@ -621,20 +816,22 @@ int orc_rdr_assign(int B, int H_kv, int64_t total_pages, const int32_t* page_off
                     s += (double)utility[e * ORC_PAGE + k];
                 U[u] = s;
                 idx[u] = e;
+                first[u] = (uint8_t)(cap ? tier_index(cap[e]) : 0);
                 forced[u] = (p < n_sink || p >= np - n_recent) ? 1 : 0;
-                if (forced[u]) forced_bytes += (int64_t)R[0];
+                if (forced[u]) forced_bytes += (int64_t)R[first[u]];
                 ++u;
             }
         }
     if (forced_bytes > budget) {
-        free(U); free(idx); free(forced);
+        free(U); free(idx); free(forced); free(first);
         return 3;
     }
 #define RDR_BYTES(lam, out_bytes)                                               \
     do {                                                                        \
         int64_t acc_ = 0;                                                       \
         for (int64_t i_ = 0; i_ < n_units; ++i_)                                \
-            acc_ += forced[i_] ? (int64_t)R[0] : (int64_t)R[rdr_choice(U[i_], eps, R, (lam))]; \
+            acc_ += forced[i_] ? (int64_t)R[first[i_]]                          \
+                               : (int64_t)R[rdr_choice(U[i_], eps, R, (lam), first[i_])]; \
         (out_bytes) = acc_;                                                     \
     } while (0)
     double lo = 0.0, hi = 1.0;
@@ -654,12 +851,12 @@ int orc_rdr_assign(int B, int H_kv, int64_t total_pages, const int32_t* page_off
     RDR_BYTES(hi, bh);
 #undef RDR_BYTES
     for (int64_t i = 0; i < n_units; ++i) {
-        int t = forced[i] ? 0 : rdr_choice(U[i], eps, R, hi);
+        int t = forced[i] ? first[i] : rdr_choice(U[i], eps, R, hi, first[i]);
         tiers[idx[i]] = (uint8_t)(t == 3 ? 0 : t + 1);
     }
     *lambda_out = hi;
     *bytes_out = bh;
-    free(U); free(idx); free(forced);
+    free(U); free(idx); free(forced); free(first);
     return 0;
 }
 

@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 
 import oracle
+from compressed_paged_kv_ada_b200 import workloads as W
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden")
 TIERS = oracle.TIER_BITS
@@ -537,7 +538,9 @@ def test_rdr_budget_monotone_and_infeasible():
         tiers, lam, nb = _rdr_small(U, int(budget), n_sink=2, n_recent=1)
         idx = [{1: 0, 2: 1, 3: 2, 0: 3}[int(x)] for x in tiers[0]]
         D = sum(float(U[u]) * EPS[i] for u, i in enumerate(idx))
-        assert nb <= budget and nb >= prev_b * 0 and D <= prev_d * (1 + 1e-12)
+        # the Lagrangian path: a larger budget lowers lambda, and bytes(lambda)
+        # is non-increasing, so the bytes chosen never drop as the budget grows
+        assert nb <= budget and nb >= prev_b and D <= prev_d * (1 + 1e-12)
         prev_b, prev_d = nb, D
     with pytest.raises(OverflowError):
         _rdr_small(U, 4160 * 3 - 1, n_sink=2, n_recent=1)
@@ -555,3 +558,286 @@ def test_rdr_ties_go_to_higher_precision():
                                        util, eps, 5 * 4160, 0, 0, 1)
     assert lam < 1e-20
     assert tiers[0].tolist() == [1] * 5 and nb == 5 * 4160
+
+
+def test_merge_partials_is_attention_over_the_union():
+    """Pin: the log-sum-exp combine of attention over disjoint key sets equals
+    attention over their union (to fp64 rounding), whatever the split, with
+    empty parts contributing nothing; every part empty gives out 0, lse -inf."""
+    rng = np.random.default_rng(31)
+    for trial in range(20):
+        n = int(rng.integers(1, 300))
+        k = rng.standard_normal((n, 128)) * rng.lognormal(0, 0.5, 128)
+        v = rng.standard_normal((n, 128))
+        q = rng.standard_normal((4, 128)) * 3.0
+        o, l = oracle.attention(k, v, q)
+        n_parts = int(rng.integers(1, 6))
+        cuts = np.sort(rng.integers(0, n + 1, n_parts - 1))
+        bounds = np.concatenate([[0], cuts, [n]])
+        perm = rng.permutation(n)   # the parts need not be contiguous
+        outs, lses = [], []
+        for a, b in zip(bounds[:-1], bounds[1:]):
+            idx = perm[a:b]
+            oo, ll = oracle.attention(k[idx], v[idx], q)
+            outs.append(oo)
+            lses.append(ll)
+        mo, ml = oracle.merge_partials(np.stack(outs), np.stack(lses))
+        assert np.abs(ml - l).max() <= 1e-12 * max(1.0, np.abs(l).max())
+        assert np.abs(mo - o).max() <= 1e-12 * max(1.0, np.abs(o).max())
+    empty_o, empty_l = oracle.attention(np.zeros((0, 128)), np.zeros((0, 128)), np.ones((2, 128)))
+    mo, ml = oracle.merge_partials(np.stack([empty_o, empty_o]), np.stack([empty_l, empty_l]))
+    assert np.all(mo == 0) and np.all(np.isneginf(ml))
+
+
+def _tiny_cache(seq_lens, H_kv=2, seed=5):
+    """An oracle-encoded mixed-tier cache (its own encoder and packer)."""
+    w = W.make("ragged64", seq_lens=seq_lens, H_kv=H_kv, H_q=4 * H_kv, seed=seed)
+    K, V = w.dense(w.seq_lens)
+    seq, pos = w.token_index(w.seq_lens)
+    table = oracle.build_page_table(w.tiers)
+    counts = [int((w.tiers == t).sum()) for t in (1, 2, 3)]
+    pools = oracle.encode_cache(K, V, seq, pos, w.page_offsets, table, counts)
+    return w, dict(B=w.B, H_q=w.H_q, H_kv=w.H_kv, page_offsets=w.page_offsets, seq_lens=w.seq_lens,
+                   page_table=table, pools=pools)
+
+
+def test_set_keep_flips_only_radius_sign_bits_and_is_reversible():
+    """Pin: the drop flag is the sign bit of the stored radius; set_keep changes
+    exactly those bits of the present tokens of kept pages, and keeping every
+    token again restores the pages byte for byte."""
+    w, c = _tiny_cache([40, 17, 33])
+    before = [p.copy() for p in c["pools"]]
+    rng = np.random.default_rng(2)
+    keep = (rng.random((w.H_kv, w.total_pages * 16)) < 0.6).astype(np.uint8)
+    oracle.set_keep(c, keep)
+    po = w.page_offsets
+    for g in range(w.H_kv):
+        for b in range(w.B):
+            for t in range(int(w.seq_lens[b])):
+                lp = po[b] + t // 16
+                e = int(c["page_table"][g, lp]) & 0xFFFFFFFF
+                tier, phys = e >> 30, e & 0x3FFFFFFF
+                if tier == 0:
+                    continue
+                off = 2 * (t % 16)
+                r_new = int(c["pools"][tier - 1][phys, off]) | int(c["pools"][tier - 1][phys, off + 1]) << 8
+                r_old = int(before[tier - 1][phys, off]) | int(before[tier - 1][phys, off + 1]) << 8
+                assert r_old & 0x8000 == 0   # the encoder never writes a negative radius
+                want = r_old | (0 if keep[g, lp * 16 + t % 16] else 0x8000)
+                assert r_new == want
+                c["pools"][tier - 1][phys, off:off + 2] = before[tier - 1][phys, off:off + 2]
+    for p, q in zip(c["pools"], before):   # nothing else changed
+        assert np.array_equal(p, q)
+    oracle.set_keep(c, np.ones_like(keep))
+    for p, q in zip(c["pools"], before):
+        assert np.array_equal(p, q)
+
+
+def test_dropped_tokens_are_exactly_deleted():
+    """Pin: attention over a cache with tokens dropped by their flag equals,
+    bit for bit, attention over the kept tokens alone (decoded the same way);
+    keeping every token changes nothing; dropping all gives out 0, lse -inf."""
+    w, c = _tiny_cache([70, 1, 45], seed=8)
+    q = np.random.default_rng(4).standard_normal((w.B, w.H_q, 128))
+    units = [(b, g) for b in range(w.B) for g in range(w.H_kv)]
+    ro0, rl0 = oracle.cache_attention(c, q, units)
+    oracle.set_keep(c, np.ones((w.H_kv, w.total_pages * 16), np.uint8))
+    ro1, rl1 = oracle.cache_attention(c, q, units)
+    assert np.array_equal(ro0, ro1) and np.array_equal(rl0, rl1)
+    keep = (np.random.default_rng(9).random((w.H_kv, w.total_pages * 16)) < 0.5).astype(np.uint8)
+    oracle.set_keep(c, keep)
+    ro, rl = oracle.cache_attention(c, q, units)
+    po = w.page_offsets
+    for i, (b, g) in enumerate(units):
+        n = int(w.seq_lens[b])
+        K, V = w.dense_rows(b, 0, n)
+        tt = np.repeat(w.tiers[g, po[b]:po[b] + (n + 15) // 16], 16)[:n]
+        kh, vh = np.zeros((n, 128)), np.zeros((n, 128))
+        for t in (1, 2, 3):
+            idx = np.nonzero(tt == t)[0]
+            if idx.size:
+                cc = oracle.encode(K[idx, g], V[idx, g], t)
+                bl, bu, _ = oracle.TIER_BITS[t]
+                kh[idx] = oracle.decode_keys(cc["leaf"], cc["up"], cc["r16"], bl, bu)
+                vh[idx] = oracle.decode_values(cc["vq"], cc["s16"])
+        sel = (tt != 0) & (keep[g, po[b] * 16 + np.arange(n)] != 0)
+        o, l = oracle.attention(kh[sel], vh[sel], q[b, 4 * g:4 * g + 4])
+        assert np.array_equal(ro[i], o) and np.array_equal(rl[i], l)
+    oracle.set_keep(c, np.zeros((w.H_kv, w.total_pages * 16), np.uint8))
+    ro, rl = oracle.cache_attention(c, q, units)
+    assert np.all(ro == 0) and np.all(np.isneginf(rl))
+
+
+# --------------------------------------------- transcode / RDR re-run pins --
+def _angle_dist_leaf(a, b):
+    d = abs(a - b) % (2 * math.pi)
+    return min(d, 2 * math.pi - d)
+
+
+@pytest.mark.parametrize("pair", [(1, 2), (1, 3), (2, 3)])
+def test_transcode_angles_are_nearest_coarse_grid_points(pair):
+    """Pin (brute force over every code): a transcoded leaf code is the
+    nearest point of the coarser periodic grid to the fine angle, ties to the
+    even code; a transcoded upper code is the nearest point of the coarser
+    end-inclusive grid (whose odd step count leaves no ties)."""
+    a, b = pair
+    bla, bua, _ = TIERS[a]
+    blb, bub, _ = TIERS[b]
+    for c in range(1 << bla):
+        phi = 2 * math.pi * c / (1 << bla)
+        dists = [_angle_dist_leaf(phi, 2 * math.pi * k / (1 << blb)) for k in range(1 << blb)]
+        best = min(dists)
+        cands = [k for k, dd in enumerate(dists) if dd <= best + 1e-12]
+        got = oracle.transcode_token(a, b, np.full(64, c, np.uint8), np.zeros(63, np.uint8), 0,
+                                     np.zeros(128, np.int8))["leaf"][0]
+        assert got in cands and (len(cands) == 1 or got % 2 == 0), (c, cands, got)
+    for c in range(1 << bua):
+        psi = (math.pi / 2) * c / ((1 << bua) - 1)
+        dists = [abs(psi - (math.pi / 2) * k / ((1 << bub) - 1)) for k in range(1 << bub)]
+        got = oracle.transcode_token(a, b, np.zeros(64, np.uint8), np.full(63, c, np.uint8), 0,
+                                     np.zeros(128, np.int8))["up"][0]
+        assert dists[got] <= min(dists) + 1e-12 and sorted(dists)[1] > min(dists) + 1e-9
+
+
+@pytest.mark.parametrize("pair", [(1, 2), (1, 3), (2, 3)])
+def test_transcode_equals_reencoding_the_decoded_token(pair):
+    """Pin: away from exact ties of the leaf grid, transcoding equals running
+    the encoder on the decoded (fp64) key and values of the finer tier; value
+    codes and scales agree always (the same fp64 quantiser on the same
+    values)."""
+    a, b = pair
+    bla, bua, _ = TIERS[a]
+    rng = np.random.default_rng(40 + a * 3 + b)
+    K = rng.standard_normal((200, 128)) * rng.lognormal(0, 0.5, 128)
+    V = rng.standard_normal((200, 128)) * np.where(rng.random((200, 1)) < 0.1, 50.0, 1.0)
+    ca = oracle.encode(K, V, a)
+    kh = oracle.decode_keys(ca["leaf"], ca["up"], ca["r16"], bla, bua)
+    vh = oracle.decode_values(ca["vq"], ca["s16"])
+    cb = oracle.encode(kh, vh, b)
+    blb, bub, _ = TIERS[b]
+    tie = (ca["leaf"].astype(np.int64) << blb) % (1 << bla) == (1 << bla) // 2
+    n_cmp = 0
+    for i in range(200):
+        tc = oracle.transcode_token(a, b, ca["leaf"][i], ca["up"][i], ca["s16"][i], ca["vq"][i])
+        # compare the keys the codes decode to: codes under a subtree whose
+        # weight is exactly 0 (an upper code 0 gives sin = 0) do not matter,
+        # and the encoder writes 0 there
+        kt = oracle.decode_keys(tc["leaf"][None], tc["up"][None], ca["r16"][i:i + 1], blb, bub)[0]
+        kr = oracle.decode_keys(cb["leaf"][i:i + 1], cb["up"][i:i + 1], cb["r16"][i:i + 1], blb, bub)[0]
+        ok = np.repeat(~tie[i], 2)
+        assert np.array_equal(kt[ok], kr[ok])
+        assert tc["s16"] == cb["s16"][i] and np.array_equal(tc["vq"], cb["vq"][i])
+        n_cmp += int(ok.sum())
+    assert n_cmp > 200 * 128 * 0.4   # T2 -> T3: every odd leaf code is a tie
+
+
+def test_transcode_direction_error_within_both_tiers_bounds():
+    """Pin (triangle inequality): a key transcoded T1 -> T3 stays within the
+    sum of the T1 and T3 worst-case angle bounds of the exact direction."""
+    rng = np.random.default_rng(44)
+    K = rng.standard_normal((300, 128)) * rng.lognormal(0, 0.5, 128)
+    V = rng.standard_normal((300, 128))
+    c1 = oracle.encode(K, V, 1)
+
+    def bound(t):
+        bl, bu, _ = TIERS[t]
+        return math.pi / 2 ** bl + 6 * (math.pi / 2) / (2 * (2 ** bu - 1))
+
+    for i in range(300):
+        tc = oracle.transcode_token(1, 3, c1["leaf"][i], c1["up"][i], c1["s16"][i], c1["vq"][i])
+        u = oracle.decode_keys(tc["leaf"][None], tc["up"][None], np.array([0x3C00], np.uint16), 3, 4)[0]
+        k = K[i] / np.linalg.norm(K[i])
+        assert np.linalg.norm(u - k) <= bound(1) + bound(3) + 1e-12
+
+
+def test_rdr_rerun_uncapped_equals_assign_and_respects_caps():
+    """Pin: with every page at T1 (nothing to cap) the re-run is RDR itself;
+    with caps, no page becomes finer than it was, forced pages keep the finest
+    tier allowed, and the bytes fit the budget."""
+    rng = np.random.default_rng(12)
+    po = np.array([0, 30, 45, 90], np.int32)
+    lens = np.array([400, 150, 600], np.int32)     # 25, 10, 38 pages of 30, 15, 45 reserved
+    util = rng.lognormal(0, 1, (2, 90 * 16)).astype(np.float32)
+    budget = 400_000
+    t_all1 = np.ones((2, 90), np.uint8)
+    a = oracle.rdr_assign(po, lens, util, EPS, budget, 4, 8, 2, tiers_init=t_all1)
+    b = oracle.rdr_rerun(po, lens, util, EPS, budget, 4, 8, t_all1)
+    assert np.array_equal(a[0], b[0]) and a[1] == b[1] and a[2] == b[2]
+    cur = a[0]
+    lens2 = lens + 40
+    new, lam, nb = oracle.rdr_rerun(po, lens2, util, EPS, 380_000, 4, 8, cur)
+    idx = lambda t: np.where(t == 0, 3, t.astype(np.int64) - 1)   # noqa: E731
+    for g in range(2):
+        for s in range(3):
+            npg = (int(lens2[s]) + 15) // 16
+            for p in range(npg):
+                e = po[s] + p
+                assert idx(new[g, e]) >= idx(cur[g, e])
+                if p < 4 or p >= npg - 8:
+                    assert new[g, e] == cur[g, e]
+    assert nb <= 380_000
+
+
+def test_rdr_rerun_brute_force_optimal_under_caps():
+    """Pin: brute force over every capped assignment (n <= 7 units): the
+    re-run's choice has the least distortion among assignments that respect
+    the caps and use no more bytes."""
+    rng = np.random.default_rng(13)
+    R = [4160, 2368, 1984, 0]
+    for trial in range(20):
+        n = int(rng.integers(2, 8))
+        util = np.zeros((1, n * 16), np.float32)
+        util[0] = rng.lognormal(0, 1.5, n * 16).astype(np.float32)
+        cur = rng.choice(np.array([1, 2, 3, 0], np.uint8), size=(1, n))
+        cidx = [3 if x == 0 else int(x) - 1 for x in cur[0]]
+        floor = sum(R[i] for i in cidx)   # every unit at its finest allowed tier
+        budget = int(rng.integers(0, floor + 1))
+        t, lam, nb = oracle.rdr_rerun(np.array([0, n], np.int32), np.array([16 * n], np.int32), util, EPS, budget,
+                                      0, 0, cur)
+        got = [3 if x == 0 else int(x) - 1 for x in t[0]]
+        U = util[0].reshape(n, 16).astype(np.float64).sum(1)
+        D = sum(U[u] * EPS[i] for u, i in enumerate(got))
+        assert sum(R[i] for i in got) == nb <= budget
+        best = math.inf
+        for combo in itertools.product(range(4), repeat=n):
+            if any(combo[u] < cidx[u] for u in range(n)):
+                continue
+            if sum(R[i] for i in combo) <= nb:
+                best = min(best, sum(U[u] * EPS[i] for u, i in enumerate(combo)))
+        assert D <= best * (1 + 1e-12) + 1e-300
+
+
+def test_migrate_moves_unchanged_pages_byte_for_byte_and_transcodes_the_rest():
+    """Pin: migrating to the same tiers reproduces every page byte for byte
+    (pool ids may differ); with coarser tiers, every token unpacked from its new
+    page equals the transcode of the token unpacked from its old page."""
+    w, c = _tiny_cache([300, 77, 160], seed=21)
+    counts = [int((w.tiers == t).sum()) for t in (1, 2, 3)]
+    perm = [np.random.default_rng(t).permutation(counts[t]).astype(np.int32) for t in range(3)]
+    table2 = oracle.build_page_table(w.tiers, perm)
+    new = oracle.migrate(c, table2, counts)
+    for t in range(3):
+        for k in range(counts[t]):
+            assert np.array_equal(new[t][perm[t][k]], c["pools"][t][k])
+    coarse = w.tiers.copy()
+    coarse[coarse == 1] = 2
+    coarse[(coarse == 2) & (np.arange(coarse.shape[1]) % 3 == 0)] = 3
+    counts2 = [int((coarse == t).sum()) for t in (1, 2, 3)]
+    table3 = oracle.build_page_table(coarse)
+    new3 = oracle.migrate(c, table3, counts2)
+    po = w.page_offsets
+    for g in range(w.H_kv):
+        for b in range(w.B):
+            for tok in range(int(w.seq_lens[b])):
+                lp = po[b] + tok // 16
+                eo, en = int(c["page_table"][g, lp]) & 0xFFFFFFFF, int(table3[g, lp]) & 0xFFFFFFFF
+                to, tn = eo >> 30, en >> 30
+                if tn == 0:
+                    continue
+                old = oracle.unpack_token(to, tok % 16, c["pools"][to - 1][eo & 0x3FFFFFFF])
+                got = oracle.unpack_token(tn, tok % 16, new3[tn - 1][en & 0x3FFFFFFF])
+                want = oracle.transcode_token(to, tn, old["leaf"], old["up"], old["s16"], old["vq"]) if tn != to else old
+                assert got["r16"] == old["r16"]
+                for f in ("leaf", "up", "vq"):
+                    assert np.array_equal(got[f], want[f])
+                assert got["s16"] == want["s16"]
