@@ -765,7 +765,8 @@ def test_rdr_rerun_uncapped_equals_assign_and_respects_caps():
     assert np.array_equal(a[0], b[0]) and a[1] == b[1] and a[2] == b[2]
     cur = a[0]
     lens2 = lens + 40
-    new, lam, nb = oracle.rdr_rerun(po, lens2, util, EPS, 380_000, 4, 8, cur)
+    # a larger budget than before: unconstrained, many pages would become finer
+    new, lam, nb = oracle.rdr_rerun(po, lens2, util, EPS, 600_000, 4, 8, cur)
     idx = lambda t: np.where(t == 0, 3, t.astype(np.int64) - 1)   # noqa: E731
     for g in range(2):
         for s in range(3):
@@ -775,7 +776,9 @@ def test_rdr_rerun_uncapped_equals_assign_and_respects_caps():
                 assert idx(new[g, e]) >= idx(cur[g, e])
                 if p < 4 or p >= npg - 8:
                     assert new[g, e] == cur[g, e]
-    assert nb <= 380_000
+    assert nb <= 600_000
+    free = oracle.rdr_assign(po, lens2, util, EPS, 600_000, 4, 8, 2, tiers_init=np.ones((2, 90), np.uint8))[0]
+    assert (idx(free) < idx(cur)).any()   # the caps did bind somewhere
 
 
 def test_rdr_rerun_brute_force_optimal_under_caps():
@@ -795,6 +798,7 @@ def test_rdr_rerun_brute_force_optimal_under_caps():
         t, lam, nb = oracle.rdr_rerun(np.array([0, n], np.int32), np.array([16 * n], np.int32), util, EPS, budget,
                                       0, 0, cur)
         got = [3 if x == 0 else int(x) - 1 for x in t[0]]
+        assert all(got[u] >= cidx[u] for u in range(n))   # no unit became finer
         U = util[0].reshape(n, 16).astype(np.float64).sum(1)
         D = sum(U[u] * EPS[i] for u, i in enumerate(got))
         assert sum(R[i] for i in got) == nb <= budget
@@ -841,3 +845,18 @@ def test_migrate_moves_unchanged_pages_byte_for_byte_and_transcodes_the_rest():
                 for f in ("leaf", "up", "vq"):
                     assert np.array_equal(got[f], want[f])
                 assert got["s16"] == want["s16"]
+
+
+def test_rdr_rerun_counts_forced_pages_at_their_capped_tier():
+    """Pin: forced pages that a re-run caps below T1 cost their own tier's
+    bytes; a budget that fits them at that tier (but not at T1) is feasible
+    and keeps them there."""
+    po = np.array([0, 12], np.int32)
+    lens = np.array([12 * 16], np.int32)
+    util = np.ones((1, 12 * 16), np.float32)
+    cur = np.full((1, 12), 3, np.uint8)        # every page T3, all forced (4 sink + 8 recent)
+    budget = 12 * 1984 + 100                   # fits 12 T3 pages, far below 12 T1 pages
+    t, lam, nb = oracle.rdr_rerun(po, lens, util, EPS, budget, 4, 8, cur)
+    assert t[0].tolist() == [3] * 12 and nb == 12 * 1984
+    with pytest.raises(OverflowError):
+        oracle.rdr_rerun(po, lens, util, EPS, 12 * 1984 - 1, 4, 8, cur)
