@@ -11,11 +11,17 @@ from ._lib import (  # noqa: F401
     make_cache,
     sphkv_build_page_table,
     sphkv_decode_attention,
+    sphkv_decode_attention_mq,
     sphkv_decode_attention_noalloc,
+    sphkv_decode_mq_workspace_bytes,
     sphkv_decode_workspace_bytes,
     sphkv_encode,
+    sphkv_merge_partials,
+    sphkv_migrate,
     sphkv_page_bytes,
     sphkv_rdr_assign,
+    sphkv_rdr_rerun,
     sphkv_rdr_workspace_bytes,
+    sphkv_set_keep,
 )
 from .cache import PagedCache  # noqa: F401

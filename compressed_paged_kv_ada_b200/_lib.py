@@ -45,7 +45,8 @@ _lib = None
 _EXPORTS = ("sphkv_page_bytes", "sphkv_last_error", "sphkv_encode", "sphkv_rdr_workspace_bytes",
             "sphkv_rdr_assign", "sphkv_build_page_table", "sphkv_decode_workspace_bytes",
             "sphkv_decode_attention", "sphkv_decode_attention_noalloc", "sphkv_decode_mq_workspace_bytes",
-            "sphkv_decode_attention_mq")
+            "sphkv_decode_attention_mq", "sphkv_merge_partials", "sphkv_set_keep", "sphkv_rdr_rerun",
+            "sphkv_migrate")
 
 
 def lib() -> ctypes.CDLL:
@@ -87,6 +88,14 @@ def load(path: str) -> ctypes.CDLL:
     L.sphkv_decode_attention_mq.restype = c.c_int
     L.sphkv_decode_attention_mq.argtypes = [c.POINTER(sphkv_cache), c.c_int32, c.c_int32, P, P, P, P,
                                             c.c_size_t, P, P]
+    L.sphkv_rdr_rerun.restype = c.c_int
+    L.sphkv_rdr_rerun.argtypes = L.sphkv_rdr_assign.argtypes
+    L.sphkv_migrate.restype = c.c_int
+    L.sphkv_migrate.argtypes = [c.POINTER(sphkv_cache), c.POINTER(sphkv_cache), P, P]
+    L.sphkv_set_keep.restype = c.c_int
+    L.sphkv_set_keep.argtypes = [c.POINTER(sphkv_cache), P, P, P]
+    L.sphkv_merge_partials.restype = c.c_int
+    L.sphkv_merge_partials.argtypes = [P, P, c.c_int32, c.c_int64, P, P, P]
     return L
 
 
@@ -162,6 +171,24 @@ def sphkv_rdr_assign(cache: sphkv_cache, utility: torch.Tensor, eps: Sequence[fl
         _ptr(status, torch.int32, "status"), _stream(stream)))
 
 
+def sphkv_rdr_rerun(cache: sphkv_cache, utility: torch.Tensor, eps: Sequence[float], budget: int,
+                    n_sink: int, n_recent: int, tiers_io: torch.Tensor, lambda_out: torch.Tensor,
+                    bytes_out: torch.Tensor, workspace: torch.Tensor,
+                    status: Optional[torch.Tensor] = None, stream=None):
+    e = (ctypes.c_double * 4)(*[float(x) for x in eps])
+    _check("sphkv_rdr_rerun", lib().sphkv_rdr_rerun(
+        ctypes.byref(cache), _ptr(utility, torch.float32, "utility"), e, int(budget), int(n_sink),
+        int(n_recent), _ptr(tiers_io, torch.uint8, "tiers_io"),
+        _ptr(lambda_out, torch.float64, "lambda_out"), _ptr(bytes_out, torch.int64, "bytes_out"),
+        _ptr(workspace, torch.uint8, "workspace"), int(workspace.numel()),
+        _ptr(status, torch.int32, "status"), _stream(stream)))
+
+
+def sphkv_migrate(src: sphkv_cache, dst: sphkv_cache, status: Optional[torch.Tensor] = None, stream=None):
+    _check("sphkv_migrate", lib().sphkv_migrate(ctypes.byref(src), ctypes.byref(dst),
+                                                _ptr(status, torch.int32, "status"), _stream(stream)))
+
+
 def sphkv_build_page_table(tiers: torch.Tensor, table: torch.Tensor, perms=(None, None, None),
                            counts: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
                            stream=None):
@@ -207,3 +234,24 @@ def sphkv_decode_attention_mq(cache: sphkv_cache, n_q: int, H_q: int, q: torch.T
         ctypes.byref(cache), int(n_q), int(H_q), _ptr(q, torch.float32, "q"), _ptr(out, torch.float32, "out"),
         _ptr(lse, torch.float32, "lse"), _ptr(workspace, torch.uint8, "workspace"),
         int(workspace.numel()), _ptr(status, torch.int32, "status"), _stream(stream)))
+
+
+def sphkv_merge_partials(out_parts: torch.Tensor, lse_parts: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
+                         stream=None):
+    """Log-sum-exp combine of decode results over disjoint parts of the same
+    sequences: out_parts [n_parts, ..., 128], lse_parts [n_parts, ...] ->
+    out [..., 128], lse [...]."""
+    n_parts = int(lse_parts.shape[0])
+    n_rows = int(lse.numel())
+    if out_parts.shape[0] != n_parts or out_parts[0].numel() != n_rows * 128 or out.numel() != n_rows * 128:
+        raise ValueError("sphkv_merge_partials: shapes do not match")
+    _check("sphkv_merge_partials", lib().sphkv_merge_partials(
+        _ptr(out_parts, torch.float32, "out_parts"), _ptr(lse_parts, torch.float32, "lse_parts"), n_parts, n_rows,
+        _ptr(out, torch.float32, "out"), _ptr(lse, torch.float32, "lse"), _stream(stream)))
+
+
+def sphkv_set_keep(cache: sphkv_cache, keep: torch.Tensor, status: Optional[torch.Tensor] = None, stream=None):
+    """Per-token keep/drop: keep [H_kv, total_pages * 16] uint8 (nonzero =
+    keep) sets or clears each present token's drop flag."""
+    _check("sphkv_set_keep", lib().sphkv_set_keep(
+        ctypes.byref(cache), _ptr(keep, torch.uint8, "keep"), _ptr(status, torch.int32, "status"), _stream(stream)))

@@ -32,6 +32,8 @@ SOURCES = {
     "encode.cu": ["-fmad=false"],
     "rdr.cu": ["-fmad=false"],
     "decode.cu": [],
+    "splitkv.cu": [],
+    "keep.cu": [],
 }
 
 

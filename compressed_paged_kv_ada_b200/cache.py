@@ -58,6 +58,11 @@ class PagedCache:
     def encode(self, K: torch.Tensor, V: torch.Tensor, tok_seq: torch.Tensor, tok_pos: torch.Tensor):
         L.sphkv_encode(self.descriptor(), K, V, tok_seq, tok_pos, status=self.status)
 
+    def set_keep(self, keep: torch.Tensor):
+        """Per-token keep/drop flags: keep [H_kv, total_pages * 16] uint8
+        (nonzero = keep), in the layout of RDR's utility."""
+        L.sphkv_set_keep(self.descriptor(), keep, status=self.status)
+
     def workspace(self, H_q: int) -> torch.Tensor:
         n = L.sphkv_decode_workspace_bytes(self.B, H_q, self.H_kv, self.total_pages)
         if self._ws is None or self._ws.numel() < n:
@@ -92,6 +97,33 @@ class PagedCache:
         nbytes = torch.zeros(1, dtype=torch.int64, device=self.device)
         L.sphkv_rdr_assign(self.descriptor(), utility, eps, budget, n_sink, n_recent, self.tiers, lam,
                            nbytes, ws, status=self.status)
+        return lam, nbytes
+
+    def rdr_rerun(self, utility: torch.Tensor, eps, budget: int, n_sink: int, n_recent: int):
+        """RDR again on the grown cache, each page capped at its current tier,
+        then the tokens transcoded into new, compacted pools (sphkv_rdr_rerun,
+        sphkv_build_page_table, sphkv_migrate).  Returns (lambda, bytes) as
+        device tensors; self.tiers, page_table and pools are replaced."""
+        ws = torch.empty(L.sphkv_rdr_workspace_bytes(self.B, self.H_kv, self.total_pages),
+                         dtype=torch.uint8, device=self.device)
+        lam = torch.zeros(1, dtype=torch.float64, device=self.device)
+        nbytes = torch.zeros(1, dtype=torch.int64, device=self.device)
+        new_tiers = self.tiers.clone()
+        L.sphkv_rdr_rerun(self.descriptor(), utility, eps, budget, n_sink, n_recent, new_tiers, lam, nbytes, ws,
+                          status=self.status)
+        self.check()
+        old = self.descriptor()
+        old_keep = (self.pools, self.page_table)   # alive until the migration has run
+        counts = [int((new_tiers == t).sum().item()) for t in (1, 2, 3)]
+        self.tiers = new_tiers
+        self.pools = [torch.zeros((counts[t], L.sphkv_page_bytes(t + 1)), dtype=torch.uint8,
+                                  device=self.device) for t in range(3)]
+        self.page_table = torch.empty((self.H_kv, self.total_pages), dtype=torch.int32, device=self.device)
+        self.perms = [None, None, None]
+        self.build_page_table()
+        L.sphkv_migrate(old, self.descriptor(), status=self.status)
+        self.check()
+        del old_keep
         return lam, nbytes
 
     def reallocate_pools(self):

@@ -44,7 +44,6 @@
 // head); decode_kernel<2> serves a pair of causal query tokens (8 heads), see
 // "two query tokens per pass" below.
 #include <cstdlib>
-#include <mutex>
 
 #include "common.cuh"
 
@@ -52,48 +51,82 @@ namespace sphkv {
 namespace {
 
 constexpr int kG = 4;               // query heads per kv head
-constexpr int kWarps = 16;
-constexpr int kThreads = kWarps * 32;
-constexpr int kStages = 2;
 constexpr int kStageBytes = Tier<1>::f.page_bytes;  // largest page
 constexpr int kMinPagesPerCta = 64;
 constexpr int kPartStride = 132;    // floats per (slot, head): m, l, pad, pad, o[128]
 
-// Cos/sin tables.  T1: one 256-byte row per code, [leaf (cos,sin) x 16 lane
-// replicas][upper (cos,sin) x 16 replicas].  T2, T3: upper grid only, one
-// 128-byte row of 16 replicas per code (their leaves are read from the
-// query-folded table below), and one unreplicated (cos,sin) per T2 leaf code
-// for building it.
-constexpr int kLutT1 = 0;                    // 256 rows x 256 B
-constexpr int kLutT2 = 256 * 256;            // 64 rows x 128 B
-constexpr int kLutT3 = kLutT2 + 64 * 128;    // 16 rows x 128 B
-constexpr int kLeafT2 = kLutT3 + 16 * 128;   // 16 x (cos, sin)
-constexpr int kLutBytes = (kLeafT2 + 16 * 8 + 127) / 128 * 128;
-constexpr int kStageOff = kLutBytes;
-constexpr int kPbufOff = kStageOff + kWarps * kStages * kStageBytes;
-constexpr int kPbufFloats = 16 * kG + 2 * kG;   // p*scale per (token, head); alpha per head; pad
-// Query-folded leaf table of the current unit on the T2 leaf grid (16 codes):
-// entry (code c, leaf j = 8s + i) holds q_h[2j] cos(phi_c) + q_h[2j+1]
-// sin(phi_c) for the 4 heads (16 bytes) at byte (c << 10) + 128 s + 16 (i ^ s):
-// the 8 lanes of a token look up the same i for different s, which lands in 8
-// distinct banks.  The T3 leaf grid (8 codes) is the even half of it: T3 code
-// c has the angle of T2 code 2c.
-constexpr int kFoldOff = (kPbufOff + kWarps * kPbufFloats * 4 + 127) / 128 * 128;
-constexpr int kFoldBytes = 16 * 1024;
-// The unit's query for T1 leaves: (q[2j], q[2j+1]) of leaf j = 8s + i for
-// heads 0, 1 and for heads 2, 3, in two 1 KB arrays of 16-byte entries at
-// byte 144 s ^ 16 i, so the 8 subtree lanes of a token read 8 distinct banks.
-constexpr int kQOff = kFoldOff + kFoldBytes;
-constexpr int kQBytes = 2 * kLeaves * 16;
-constexpr int kBarOff = kQOff + kQBytes;
-constexpr int kSliceOff = kBarOff + kWarps * kStages * 8;   // per-warp slice weights
-constexpr int kSmemBytes = kSliceOff + kWarps * 4;
-static_assert(kStageOff % 128 == 0 && kPbufOff % 16 == 0 && kFoldOff % 128 == 0 && kQOff % 128 == 0 &&
-                  kBarOff % 8 == 0,
-              "smem alignment");
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-// CTA merge scratch (aliases the stage ring): m[16][4], l[16][4], o[16][4][128]
-static_assert((2 * kWarps * kG + kWarps * kG * kD) * 4 <= kWarps * kStages * kStageBytes, "merge scratch");
+// Cos/sin tables, shared by both decode kernels.  T1: one 256-byte row per
+// code, [leaf (cos,sin) x 16 lane replicas][upper (cos,sin) x 16 replicas].
+// T2, T3: upper grid only, one 128-byte row of 16 replicas per code.  T2 and
+// T3 leaves read T1 leaf rows or the query-folded table: the leaf grids nest
+// (T2 code c has the angle of T1 code 16c, T3 code c that of T2 code 2c).
+//
+// Shared-memory layout of decode_kernel<NQ>.  Region offsets are taken from a
+// zero point: for one query token (NQ = 1) that is shared address 0, i.e. the
+// offsets are absolute shared-window addresses, each table aligned to its own
+// size so that a lookup address is the OR of the table base, the code and the
+// lane's replica (one instruction per code, no address add); the dynamic block
+// must then start below the first region, which the kernel checks.  For a pair
+// of query tokens (NQ = 2) the zero point is the start of the dynamic block.
+template <int NQ>
+struct Layout;
+// One query token: 12 warps, 8 lanes per token, each lane holding its
+// subtree's query slice in registers (168 registers a thread); two-stage page
+// rings.  The query-folded T2/T3 leaf table holds, for leaf j = 8s + i and T2
+// code c, the 4 heads' q[2j] cos(phi_c) + q[2j+1] sin(phi_c) (times the logit
+// scale) at kFold + (c << 11) + 144 s + 16 i, in the head order of the lanes
+// that own subtree s.
+template <>
+struct Layout<1> {
+    static constexpr int kWarps = 12;
+    static constexpr int kStages = 2;
+    static constexpr int kHeads = kG;
+    static constexpr int kPbufFloats = 16 * kG + 2 * kG;   // p*scale per (token, head); alpha per head; valid
+    static constexpr uint32_t kUpT2 = 8192;                // 64 rows x 128 B, 8 KB aligned
+    static constexpr uint32_t kUpT3 = 16384;               // 16 rows x 128 B, 2 KB aligned
+    static constexpr uint32_t kPbuf = 18432;
+    static constexpr uint32_t kBar = kPbuf + kWarps * kPbufFloats * 4;
+    static constexpr uint32_t kSlice = kBar + kWarps * kStages * 8;
+    static constexpr uint32_t kFold = 32768;               // 16 codes x 2 KB, 32 KB aligned
+    static constexpr uint32_t kT1 = 65536;                 // 256 rows x 256 B, 64 KB aligned
+    static constexpr uint32_t kStage = 131072;
+    static constexpr int kSmemBytes = (int)(kStage + kWarps * kStages * kStageBytes);
+};
+// A pair of query tokens (8 heads): 16 warps, two-stage rings; the pair's
+// query rows (4 arrays of (q[2j], q[2j+1]) for heads 2a, 2a+1, at byte
+// 1024 a + (144 s ^ 16 i) for leaf j = 8s + i) sit in shared memory.
+template <>
+struct Layout<2> {
+    static constexpr int kWarps = 16;
+    static constexpr int kStages = 2;
+    static constexpr int kHeads = 2 * kG;
+    static constexpr int kPbufFloats = 16 * 2 * kG + 2 * 2 * kG;   // weights; alpha; valid counts
+    static constexpr uint32_t kT1 = 0;
+    static constexpr uint32_t kUpT2 = 256 * 256;
+    static constexpr uint32_t kUpT3 = kUpT2 + 64 * 128;
+    static constexpr uint32_t kStage = kUpT3 + 16 * 128;
+    static constexpr uint32_t kQ = kStage + kWarps * kStages * kStageBytes;
+    static constexpr uint32_t kPbuf = kQ + 4 * 1024;
+    static constexpr uint32_t kBar = kPbuf + kWarps * kPbufFloats * 4;
+    static constexpr uint32_t kSlice = kBar + kWarps * kStages * 8;
+    static constexpr int kSmemBytes = (int)(kSlice + kWarps * 4);
+};
+constexpr int kLutT1 = 0, kLutT2 = Layout<2>::kUpT2, kLutT3 = Layout<2>::kUpT3;   // pair kernel, relative
+template <int NQ>
+constexpr bool layout_ok()
+{
+    using L = Layout<NQ>;
+    return L::kStage % 128 == 0 && L::kPbuf % 16 == 0 && L::kBar % 8 == 0 && L::kT1 % 65536 == 0 &&
+           L::kUpT2 % 8192 == 0 && L::kUpT3 % 2048 == 0 && L::kSmemBytes <= 227 * 1024 &&
+           // CTA merge scratch (aliases the rings): m[W][H], l[W][H], o[W][H][128]
+           (2 * L::kWarps * L::kHeads + L::kWarps * L::kHeads * kD) * 4 <=
+               L::kWarps * L::kStages * kStageBytes;
+}
+static_assert(layout_ok<1>() && layout_ok<2>(), "shared-memory layout");
+static_assert(Layout<1>::kSlice + Layout<1>::kWarps * 4 <= Layout<1>::kFold && Layout<1>::kFold % 32768 == 0 &&
+                  Layout<1>::kFold + 32768 <= Layout<1>::kT1 && Layout<1>::kT1 + 65536 <= Layout<1>::kStage,
+              "one-query regions");
+static_assert(Layout<2>::kQ % 128 == 0, "pair query rows");
 
 constexpr float kLn2 = 0.6931471805599453f;
 // log2(e) / sqrt(128): logits are kept in the log2 domain
@@ -123,8 +156,9 @@ struct DecodeParams {
     int nq, q0, npair, len_shift;
 #ifdef SPHKV_TEST_HOOKS
     // Test builds only (environment SPHKV_TEST_SKIP_FIRST_COPY): warp 0 of
-    // CTA 0 skips its first page copy, so its bounded wait runs out (after a
-    // short limit) and the call reports SPHKV_ERR_TIMEOUT without any fault.
+    // CTA 0 skips its first page copy and waits with a short limit, so that
+    // wait runs out and the call reports SPHKV_ERR_TIMEOUT without any fault;
+    // every other warp and CTA runs as in the product build.
     int test_skip_copy;
 #endif
     const float* q;
@@ -293,45 +327,52 @@ __device__ __forceinline__ float pow2_floor(float x)
     return __int_as_float(__float_as_int(x) & 0x7f800000);
 }
 
-// Offsets of the 8 leaf and 8 upper codes of one subtree block.  T1: byte
-// offset code << 8 | replica << 3 into its 256-byte rows; T2/T3 upper codes:
-// code << 7 | replica << 3; base_rep = (lane & 15) << 3.  T2/T3 leaves: offset
-// (T3 code c read as T2 code 2c) into the query-folded table,
-// code << 10 | fl[i] for leaf i of subtree s, fl[i] = 144 s ^ 16 i.
+// Table offsets of the 8 leaf and 8 upper codes of one subtree block.  Leaves
+// (every tier) index T1 leaf rows: T1 code c at c << 8, T2 code c at c << 12
+// (T1 row 16c), T3 code c at c << 13 (T1 row 32c).  Upper codes: T1 c << 8
+// (the upper half is 128 bytes into the row), T2/T3 c << 7 into their own
+// 128-byte rows.  rep = (lane & 15) << 3 picks the lane's replica, so a half
+// warp's 64-bit lookups never share a bank.
 template <int T>
-__device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uint32_t base_rep,
-                                              const uint32_t (&fl)[8], uint32_t (&lo)[8], uint32_t (&uo)[8])
+__device__ __forceinline__ uint32_t shift_mask(uint32_t x, int sh, uint32_t mask)
+{
+    return (sh >= 0 ? x << sh : x >> -sh) & mask;
+}
+
+template <int T>
+__device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uint32_t rep, uint32_t (&lo)[8],
+                                              uint32_t (&uo)[8])
 {
     if (T == 1) {   // byte codes: one permute places the code in bits 8..15
         const uint4 w = *(const uint4*)(codes + blk * 16);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            lo[j] = __byte_perm(w.x, base_rep, 0x7604 | (j << 4));
-            lo[4 + j] = __byte_perm(w.y, base_rep, 0x7604 | (j << 4));
-            uo[j] = __byte_perm(w.z, base_rep, 0x7604 | (j << 4));
-            uo[4 + j] = __byte_perm(w.w, base_rep, 0x7604 | (j << 4));
+            lo[j] = __byte_perm(w.x, rep, 0x7604 | (j << 4));
+            lo[4 + j] = __byte_perm(w.y, rep, 0x7604 | (j << 4));
+            uo[j] = __byte_perm(w.z, rep, 0x7604 | (j << 4));
+            uo[4 + j] = __byte_perm(w.w, rep, 0x7604 | (j << 4));
         }
-    } else if (T == 2) {   // upper code j = bits 6j..6j+5 of the 48-bit field h:w.y
+    } else if (T == 2) {   // leaf nibbles; upper code j = bits 6j..6j+5 of the 48-bit field h:w.y
         const uint2 w = *(const uint2*)(codes + blk * 8);
         const uint32_t h = *(const uint16_t*)(codes + kP * 64 + blk * 2);
         constexpr uint32_t kUpMask = 63u << 7;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) lo[j] = (((w.x >> (4 * j)) & 15u) << 10) | fl[j];
-        uo[0] = ((w.y << 7) & kUpMask) | base_rep;
-        uo[1] = ((w.y << 1) & kUpMask) | base_rep;
-        uo[2] = ((w.y >> 5) & kUpMask) | base_rep;
-        uo[3] = ((w.y >> 11) & kUpMask) | base_rep;
-        uo[4] = ((w.y >> 17) & kUpMask) | base_rep;
-        uo[5] = (__funnelshift_r(w.y, h, 23) & kUpMask) | base_rep;
-        uo[6] = ((h << 3) & kUpMask) | base_rep;
-        uo[7] = ((h >> 3) & kUpMask) | base_rep;
-    } else {   // leaf code j = bits 3j..3j+2 of the 24-bit field l8:l16
+        for (int j = 0; j < 8; ++j) lo[j] = shift_mask<T>(w.x, 12 - 4 * j, 15u << 12) | rep;
+        uo[0] = ((w.y << 7) & kUpMask) | rep;
+        uo[1] = ((w.y << 1) & kUpMask) | rep;
+        uo[2] = ((w.y >> 5) & kUpMask) | rep;
+        uo[3] = ((w.y >> 11) & kUpMask) | rep;
+        uo[4] = ((w.y >> 17) & kUpMask) | rep;
+        uo[5] = (__funnelshift_r(w.y, h, 23) & kUpMask) | rep;
+        uo[6] = ((h << 3) & kUpMask) | rep;
+        uo[7] = ((h >> 3) & kUpMask) | rep;
+    } else {   // upper nibbles; leaf code j = bits 3j..3j+2 of the 24-bit field l8:l16
         const uint32_t u = *(const uint32_t*)(codes + blk * 4);
         const uint32_t lf = *(const uint16_t*)(codes + kP * 32 + blk * 2) | ((uint32_t)codes[kP * 48 + blk] << 16);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            lo[j] = (((lf >> (3 * j)) & 7u) << 11) | fl[j];
-            uo[j] = (((u >> (4 * j)) & 15u) << 7) | base_rep;
+            lo[j] = shift_mask<T>(lf, 13 - 3 * j, 7u << 13) | rep;
+            uo[j] = shift_mask<T>(u, 7 - 4 * j, 15u << 7) | rep;
         }
     }
 }
@@ -369,137 +410,200 @@ __device__ __forceinline__ uint32_t block_top(const uint8_t* codes, int blk, uin
     return (((*(const uint32_t*)(codes + blk * 4)) >> 28) << 7) | base_rep;
 }
 
-// One subtree block of a token, top down from its weight v (the product of
-// the radius, the logit scale and the factors of its three ancestors):
-// accumulates the block's per-head sums (T1 in f32x2 (even, odd) pairs,
-// T2/T3 in f32x2 head pairs).
-template <int T>
-__device__ __forceinline__ void subtree(float v, const uint32_t (&lo)[8], const uint32_t (&uo)[8],
-                                        const uint8_t* smem, const uint8_t* lut, const uint8_t* lut_up,
-                                        const uint32_t (&fl)[8], float2 (&acc2)[kG], bool first)
+// Shared-memory loads by 32-bit shared address (the lookups below build full
+// addresses; these keep the compiler from adding a base to each).
+__device__ __forceinline__ float lds32(uint32_t a)
 {
-    float w2[2], w1[4], wl[8];
-    {
-        const float2 f = *(const float2*)(lut_up + uo[6]);
-        w2[0] = v * f.x;
-        w2[1] = v * f.y;
-    }
+    float v;
+    asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+    return v;
+}
+template <int Off = 0>
+__device__ __forceinline__ float2 lds64(uint32_t a)
+{
+    float2 v;
+    asm("ld.shared.v2.f32 {%0, %1}, [%2+%3];" : "=f"(v.x), "=f"(v.y) : "r"(a), "n"(Off));
+    return v;
+}
+template <int Off = 0>
+__device__ __forceinline__ float4 lds128(uint32_t a)
+{
+    float4 v;
+    asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4+%5];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a), "n"(Off));
+    return v;
+}
+
+// Full shared addresses of the 8 leaf and 8 upper lookups of one subtree
+// block, for the one-query layout.  rep1 = kT1 | leaf replica, repU = the
+// tier's upper table (kT1 for T1) | upper replica, fb = kFold | 144 s.  T1:
+// row addresses (the upper half of a row is 128 bytes on).  T2/T3 leaves: the query-folded entry of
+// leaf 0 of the block for that code (leaf i is 16 i bytes on; T3 code c is
+// T2 code 2c).
+template <int T>
+__device__ __forceinline__ void block_addrs(const uint8_t* codes, int blk, uint32_t rep1, uint32_t repU,
+                                            uint32_t fb, uint32_t (&lo)[8], uint32_t (&uo)[8])
+{
+    if (T == 1) {   // byte codes: one permute places the code in bits 8..15 under the base
+        const uint4 w = *(const uint4*)(codes + blk * 16);
 #pragma unroll
-    for (int n = 0; n < 2; ++n) {
-        const float2 f = *(const float2*)(lut_up + uo[4 + n]);
-        w1[2 * n] = w2[n] * f.x;
-        w1[2 * n + 1] = w2[n] * f.y;
-    }
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const float2 f = *(const float2*)(lut_up + uo[m]);
-        wl[2 * m] = w1[m] * f.x;
-        wl[2 * m + 1] = w1[m] * f.y;
-    }
-    if (T == 1) {   // (q[2j], q[2j+1]) . (w cos phi, w sin phi) per head
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float2 f = *(const float2*)(lut + lo[j]);
-            const float2 kk = make_float2(wl[j] * f.x, wl[j] * f.y);
-            const float4 qa = *(const float4*)(smem + kQOff + fl[j]);          // heads 0, 1
-            const float4 qb = *(const float4*)(smem + kQOff + 1024 + fl[j]);   // heads 2, 3
-            const float2 qh[kG] = {make_float2(qa.x, qa.y), make_float2(qa.z, qa.w), make_float2(qb.x, qb.y),
-                                   make_float2(qb.z, qb.w)};
-#pragma unroll
-            for (int h = 0; h < kG; ++h)
-                acc2[h] = (first && j == 0) ? __fmul2_rn(qh[h], kk) : __ffma2_rn(qh[h], kk, acc2[h]);
+        for (int j = 0; j < 4; ++j) {
+            lo[j] = __byte_perm(w.x, rep1, 0x7604 | (j << 4));
+            lo[4 + j] = __byte_perm(w.y, rep1, 0x7604 | (j << 4));
+            uo[j] = __byte_perm(w.z, repU, 0x7604 | (j << 4));
+            uo[4 + j] = __byte_perm(w.w, repU, 0x7604 | (j << 4));
         }
-    } else {   // leaf terms already folded with the query
+    } else if (T == 2) {   // leaf nibbles; upper code j = bits 6j..6j+5 of the 48-bit field h:w.y
+        const uint2 w = *(const uint2*)(codes + blk * 8);
+        const uint32_t h = *(const uint16_t*)(codes + kP * 64 + blk * 2);
+        constexpr uint32_t kUpMask = 63u << 7;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) lo[j] = shift_mask<T>(w.x, 11 - 4 * j, 15u << 11) | fb;
+        uo[0] = ((w.y << 7) & kUpMask) | repU;
+        uo[1] = ((w.y << 1) & kUpMask) | repU;
+        uo[2] = ((w.y >> 5) & kUpMask) | repU;
+        uo[3] = ((w.y >> 11) & kUpMask) | repU;
+        uo[4] = ((w.y >> 17) & kUpMask) | repU;
+        uo[5] = (__funnelshift_r(w.y, h, 23) & kUpMask) | repU;
+        uo[6] = ((h << 3) & kUpMask) | repU;
+        uo[7] = ((h >> 3) & kUpMask) | repU;
+    } else {   // upper nibbles; leaf code j = bits 3j..3j+2 of the 24-bit field l8:l16
+        const uint32_t u = *(const uint32_t*)(codes + blk * 4);
+        const uint32_t lf = *(const uint16_t*)(codes + kP * 32 + blk * 2) | ((uint32_t)codes[kP * 48 + blk] << 16);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const float4 F = *(const float4*)(smem + kFoldOff + lo[j]);
-            const float2 ww = make_float2(wl[j], wl[j]);
-            acc2[0] = (first && j == 0) ? __fmul2_rn(ww, make_float2(F.x, F.y))
-                                        : __ffma2_rn(ww, make_float2(F.x, F.y), acc2[0]);
-            acc2[1] = (first && j == 0) ? __fmul2_rn(ww, make_float2(F.z, F.w))
-                                        : __ffma2_rn(ww, make_float2(F.z, F.w), acc2[1]);
+            lo[j] = shift_mask<T>(lf, 12 - 3 * j, 7u << 12) | fb;
+            uo[j] = shift_mask<T>(u, 7 - 4 * j, 15u << 7) | repU;
         }
     }
 }
 
-// Logits of the 16 tokens of one page of tier T staged at `pg`, written in the
-// log2 domain to pbuf[t * kG + head].  Lane (k8, q), q = lane & 3, handles
-// the two subtree blocks 2q, 2q+1 (the subtree of level-4 node q) of tokens
-// 8 pass + k8 for all 4 heads, top down: the tree's value r S_root is the sum
-// over leaves of (product of the factors on the leaf's path: cos(psi) into a
-// left child, sin(psi) into a right one) times the leaf term q[2j] cos(phi_j)
-// + q[2j+1] sin(phi_j).  The path products do not depend on the head, so the
-// per-head work is one multiply-add per leaf (T2/T3, whose leaf terms are read
-// from the query-folded table) or per dimension (T1).  Odd tokens take block
-// 2q+1 first, so the 8 lanes of a quarter warp read 8 different subtrees'
-// table rows (8 distinct banks).
+// Logits of the 16 tokens of one page of tier T staged at `pg`, in the log2
+// domain: lane (k4, s) ends with lg[pass] = the logit of token 4 pass + k4 for
+// head 2 b2 + b1 (s = 4 b2 + 2 b1 + b0).  Eight lanes per token, four tokens per
+// pass: lane (k4, s) = (lane >> 3, lane & 7) evaluates subtree s (leaves
+// 8s..8s+7, the level-3 node s and the six upper nodes below it) of token
+// 4 pass + k4 for all 4 query heads, top down: the tree's value r S_root is
+// the sum over leaves of (product of the factors on the leaf's path: cos(psi)
+// into a left child, sin(psi) into a right one) times the leaf term
+// q[2j] cos(phi_j) + q[2j+1] sin(phi_j).  The three ancestors above level 3
+// (level-4 node s/2, level-5 node s/4, the root) are the top codes held in
+// slot 7 of blocks s/2, 4 + s/4 and 6, fetched by shuffles; each lane reads
+// only the factor on its own side.  The path products do not depend on the
+// head.  T1 leaves: (cos, sin) from the table times the path weight, then one
+// packed multiply-add per head with the lane's query slice (q[16s..16s+15] of
+// the 4 heads, logit scale included) in registers.  T2/T3 leaves: one 16-byte
+// lookup of the unit's query-folded table, two packed multiply-adds.  Both
+// keep the heads in the lane's slot order (slot i holds head ((i >> 1) ^ b2)
+// * 2 + ((i & 1) ^ b1) for s = 4 b2 + 2 b1 + b0), which makes the 8-lane sum
+// a select-free reduce-scatter that leaves head 2 b2 + b1 in lanes b0 = 0, 1.
 template <int T>
-__device__ __forceinline__ void page_logits(const uint8_t* pg, const uint8_t* smem, float* pbuf, int lane,
-                                            const uint32_t (&flA)[8])
+__device__ __forceinline__ void page_logits(const uint8_t* pg, int lane, const float2 (&qp)[kG][8], float (&lg)[4])
 {
+    using L = Layout<1>;
     const unsigned full = 0xffffffffu;
-    const int q = lane & 3, k8 = lane >> 2;
-    const bool a_right = k8 & 1;            // block A = 2q + 1 (right child of level-4 node q)
-    const int sA = 2 * q + (k8 & 1), sB = sA ^ 1;
-    constexpr int kBase = T == 1 ? kLutT1 : T == 2 ? kLutT2 : kLutT3;
-    constexpr int kUp = T == 1 ? 128 : 0;   // upper (cos, sin) inside a row
-    const uint8_t* lut = smem + kBase;
-    const uint8_t* lut_up = lut + kUp;
+    const int s = lane & 7;
     const uint32_t rep = (uint32_t)(lane & 15) << 3;
+    const uint32_t rep1 = L::kT1 | rep;
+    const uint32_t repU = (T == 1 ? L::kT1 : T == 2 ? L::kUpT2 : L::kUpT3) | rep;
+    const uint32_t fb = L::kFold | (144u * (uint32_t)s);
+    constexpr int kUp = T == 1 ? 128 : 0;   // upper (cos, sin) inside a T1 row
+    // own side at levels 4, 5 and the root (the upper half of a T1 row)
+    const uint32_t side4 = kUp + ((uint32_t)(s & 1) << 2), side5 = kUp + ((uint32_t)((s >> 1) & 1) << 2),
+                   side6 = kUp + ((uint32_t)(s >> 2) << 2);
+    const int grp = lane & ~7;
     const uint8_t* codes = pg + Tier<1>::f.off_codes;
-    uint32_t flB[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) flB[i] = flA[i] ^ 144u;   // 144 sB ^ 16 i
-    // ancestors: the root (level-5 node q>>1 is its left child for q < 2) and
-    // level-5 node q>>1 (level-4 node q is its left child for even q)
-    const uint32_t side6 = (uint32_t)(q >> 1) << 2, side5 = (uint32_t)(q & 1) << 2;
-    const int base = lane & ~3;
-#pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-        const int t = pass * 8 + k8;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int t = pass * 4 + (lane >> 3);
         uint32_t lo[8], uo[8];
-        block_offsets<T>(codes, t * 8 + sA, rep, flA, lo, uo);
-        const uint32_t topB = block_top<T>(codes, t * 8 + sB, rep);
-        // top codes: block i's slot 7 is top node i (level-4 nodes 0..3,
-        // level-5 nodes 0..1, root).  This lane has those of blocks 2q, 2q+1,
-        // as two 16-bit table offsets.
-        const uint32_t top2 = (a_right ? topB : uo[7]) | ((a_right ? uo[7] : topB) << 16);
-        const uint32_t w4 = __shfl_sync(full, top2, base + (q >> 1));   // block q
-        const uint32_t w5 = __shfl_sync(full, top2, base + 2);          // block 4 + (q >> 1)
-        const uint32_t w6 = __shfl_sync(full, top2, base + 3);          // block 6
-        const uint32_t o4 = (w4 >> (16 * (q & 1))) & 0xffffu;
-        const uint32_t o5 = (w5 >> (16 * (q >> 1))) & 0xffffu;
-        const uint32_t o6 = w6 & 0xffffu;
-        float v = __half2float(((const __half*)pg)[t]) * kLogitScale;
-        v *= *(const float*)(lut_up + o6 + side6);
-        v *= *(const float*)(lut_up + o5 + side5);
-        const float2 f4 = *(const float2*)(lut_up + o4);
-        const float vA = v * (a_right ? f4.y : f4.x), vB = v * (a_right ? f4.x : f4.y);
-        float2 acc2[kG];
-        subtree<T>(vA, lo, uo, smem, lut, lut_up, flA, acc2, true);
-        block_offsets<T>(codes, t * 8 + sB, rep, flB, lo, uo);
-        subtree<T>(vB, lo, uo, smem, lut, lut_up, flB, acc2, false);
-        float acc[kG];
-        if (T == 1) {
-#pragma unroll
-            for (int h = 0; h < kG; ++h) acc[h] = acc2[h].x + acc2[h].y;
-        } else {
-            acc[0] = acc2[0].x; acc[1] = acc2[0].y; acc[2] = acc2[1].x; acc[3] = acc2[1].y;
+        block_addrs<T>(codes, pass * 32 + lane, rep1, repU, fb, lo, uo);
+        // ancestors: top node s/2 (level 4), 4 + s/4 (level 5), 6 (root)
+        const uint32_t o4 = __shfl_sync(full, uo[7], grp + (s >> 1));
+        const uint32_t o5 = __shfl_sync(full, uo[7], grp + 4 + (s >> 2));
+        const uint32_t o6 = __shfl_sync(full, uo[7], grp + 6);
+        // radius bits: the sign bit is the token's drop flag, the rest the radius
+        const uint32_t rb = ((const uint16_t*)pg)[t];
+        float v = __half2float(__ushort_as_half((unsigned short)(rb & 0x7fffu)));
+        v *= lds32(o6 | side6);
+        v *= lds32(o5 | side5);
+        v *= lds32(o4 | side4);
+        float w2[2], w1[4], wl[8];
+        {
+            const float2 f = lds64<kUp>(uo[6]);
+            w2[0] = v * f.x;
+            w2[1] = v * f.y;
         }
-        // sum over the token's 4 lanes; lane q ends with head q
-        const bool b1 = q >> 1, b0 = q & 1;
-        const float x0 = (b1 ? acc[2] : acc[0]) + __shfl_xor_sync(full, b1 ? acc[0] : acc[2], 2);
-        const float x1 = (b1 ? acc[3] : acc[1]) + __shfl_xor_sync(full, b1 ? acc[1] : acc[3], 2);
-        const float y = (b0 ? x1 : x0) + __shfl_xor_sync(full, b0 ? x0 : x1, 1);
-        pbuf[t * kG + q] = y;
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+            const float2 f = lds64<kUp>(uo[4 + n]);
+            w1[2 * n] = w2[n] * f.x;
+            w1[2 * n + 1] = w2[n] * f.y;
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float2 f = lds64<kUp>(uo[m]);
+            wl[2 * m] = w1[m] * f.x;
+            wl[2 * m + 1] = w1[m] * f.y;
+        }
+        float a[kG];
+        if (T == 1) {
+            float2 acc[kG];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float2 f = lds64(lo[j]);
+                const float2 kk = make_float2(wl[j] * f.x, wl[j] * f.y);
+#pragma unroll
+                for (int i = 0; i < kG; ++i)
+                    acc[i] = j == 0 ? __fmul2_rn(qp[i][j], kk) : __ffma2_rn(qp[i][j], kk, acc[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < kG; ++i) a[i] = acc[i].x + acc[i].y;
+        } else {
+            float2 acc01, acc23;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float4 F;
+                switch (j) {   // leaf j of the block is 16 j bytes on
+                case 0: F = lds128<0>(lo[j]); break;
+                case 1: F = lds128<16>(lo[j]); break;
+                case 2: F = lds128<32>(lo[j]); break;
+                case 3: F = lds128<48>(lo[j]); break;
+                case 4: F = lds128<64>(lo[j]); break;
+                case 5: F = lds128<80>(lo[j]); break;
+                case 6: F = lds128<96>(lo[j]); break;
+                default: F = lds128<112>(lo[j]); break;
+                }
+                const float2 ww = make_float2(wl[j], wl[j]);
+                acc01 = j == 0 ? __fmul2_rn(ww, make_float2(F.x, F.y)) : __ffma2_rn(ww, make_float2(F.x, F.y), acc01);
+                acc23 = j == 0 ? __fmul2_rn(ww, make_float2(F.z, F.w)) : __ffma2_rn(ww, make_float2(F.z, F.w), acc23);
+            }
+            a[0] = acc01.x;
+            a[1] = acc01.y;
+            a[2] = acc23.x;
+            a[3] = acc23.y;
+        }
+        const float r0 = a[0] + __shfl_xor_sync(full, a[2], 4);
+        const float r1 = a[1] + __shfl_xor_sync(full, a[3], 4);
+        const float x = r0 + __shfl_xor_sync(full, r1, 2);
+        // rotate: after the last pass lg[i] holds pass i
+        lg[0] = lg[1];
+        lg[1] = lg[2];
+        lg[2] = lg[3];
+        const float y = x + __shfl_xor_sync(full, x, 1);
+        lg[3] = (rb & 0x8000u) ? -INFINITY : y;
     }
 }
 
 // Values on the tensor cores for one staged page: out^T[dims x heads] +=
 // V^T[dims x 16 tokens] P^T[16 x GQ heads], with the weights P already in
 // pbuf[t * GQ + head] and the per-head rescale factor at pbuf[16 GQ + head].
-// Thread (g, c): B columns = head g (g < GQ), rows = tokens 2c, 2c+1 (b0) and
-// 2c+8, 2c+9 (b1); accumulator columns = heads 2c, 2c+1 (mod GQ).
+// The weights are split into f16 hi + lo parts.  Four heads (one query token):
+// column n holds the hi parts of head n for n < 4 and the lo parts of head
+// n - 4 for n >= 4, so one MMA per tile takes both, and the two halves of the
+// accumulator are summed at the end (lanes c and c ^ 2).  Eight heads: the hi
+// and lo parts go through two MMAs into the same accumulator.
+// Thread (g, c): B column g, rows = tokens 2c, 2c+1 (b0) and 2c+8, 2c+9 (b1);
+// accumulator columns = heads 2c, 2c+1 (mod GQ).
 template <int GQ>
 __device__ __forceinline__ void page_values(const uint8_t* pg, int tier, const float* pbuf, int lane, float alpha_acc,
                                             WarpState& st)
@@ -516,15 +620,21 @@ __device__ __forceinline__ void page_values(const uint8_t* pg, int tier, const f
             st.acc[m][3] *= al.y;
         }
     }
+    constexpr bool kSplit = GQ == kG;   // hi and lo parts side by side in one tile
     uint32_t bh0 = 0, bh1 = 0, bl0 = 0, bl1 = 0;
-    if (g < GQ) {
-        const float p0 = pbuf[(2 * c) * GQ + g], p1 = pbuf[(2 * c + 1) * GQ + g];
-        const float p2 = pbuf[(2 * c + 8) * GQ + g], p3 = pbuf[(2 * c + 9) * GQ + g];
+    if (kSplit || g < GQ) {
+        const int hg = g % GQ;
+        const float p0 = pbuf[(2 * c) * GQ + hg], p1 = pbuf[(2 * c + 1) * GQ + hg];
+        const float p2 = pbuf[(2 * c + 8) * GQ + hg], p3 = pbuf[(2 * c + 9) * GQ + hg];
         const __half2 h01 = __floats2half2_rn(p0, p1), h23 = __floats2half2_rn(p2, p3);
         bh0 = *(const uint32_t*)&h01;
         bh1 = *(const uint32_t*)&h23;
         bl0 = pack_h2(p0 - __low2float(h01), p1 - __high2float(h01));
         bl1 = pack_h2(p2 - __low2float(h23), p3 - __high2float(h23));
+        if (kSplit && g >= GQ) {
+            bh0 = bl0;
+            bh1 = bl1;
+        }
     }
     // rows of tokens 2c, 2c+1, 2c+8, 2c+9 at positions 16g..16g+15; tokens past
     // `valid` carry weight 0 (their rows may hold anything finite)
@@ -560,7 +670,7 @@ __device__ __forceinline__ void page_values(const uint8_t* pg, int tier, const f
                 a[i] = *(const uint32_t*)&hv;
             }
             mma_16816(st.acc[m], a, bh0, bh1);
-            mma_16816(st.acc[m], a, bl0, bl1);
+            if (!kSplit) mma_16816(st.acc[m], a, bl0, bl1);
         }
     } else {   // T2 and T3 share the int4 row format
         const uint8_t* vrow = pg + (tier == 2 ? Tier<2>::f.off_v : Tier<3>::f.off_v);
@@ -598,7 +708,7 @@ __device__ __forceinline__ void page_values(const uint8_t* pg, int tier, const f
                 a[i + 1] = *(const uint32_t*)&hi;
             }
             mma_16816(st.acc[m], a, bh0, bh1);
-            mma_16816(st.acc[m], a, bl0, bl1);
+            if (!kSplit) mma_16816(st.acc[m], a, bl0, bl1);
         }
     }
 }
@@ -606,30 +716,27 @@ __device__ __forceinline__ void page_values(const uint8_t* pg, int tier, const f
 // One page of tier `tier` already staged in shared memory at `pg`.  The logits
 // are tier-specialised; the softmax and the value MMAs are one copy of code
 // for all tiers apart from the value conversion.
-__device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int valid, const uint8_t* smem, float* pbuf,
-                                             int lane, const uint32_t (&fl)[8], WarpState& st)
+__device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int valid, float* pbuf, int lane,
+                                             const float2 (&qp)[kG][8], WarpState& st)
 {
     const unsigned full = 0xffffffffu;
     const int k = lane >> 3, s = lane & 7;
-    const int head = (s & 1) * 2 + ((s >> 1) & 1);
-    // `valid` waits in the buffer's spare word while the logits hold the registers
-    if (lane == 0) ((int*)pbuf)[16 * kG + kG] = valid;
-    if (tier == 1) page_logits<1>(pg, smem, pbuf, lane, fl);
-    else if (tier == 2) page_logits<2>(pg, smem, pbuf, lane, fl);
-    else page_logits<3>(pg, smem, pbuf, lane, fl);
-    __syncwarp();
-    valid = ((const int*)pbuf)[16 * kG + kG];
-    float lg[4];
+    const int head = (s >> 2) * 2 + ((s >> 1) & 1);   // lanes b0 = 0, 1 hold the same head
+    float lg[4];   // tokens 4 pass + k of this lane's head
+    if (tier == 1) page_logits<1>(pg, lane, qp, lg);
+    else if (tier == 2) page_logits<2>(pg, lane, qp, lg);
+    else page_logits<3>(pg, lane, qp, lg);
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass)   // slots past `valid` (last page) get -inf
-        lg[pass] = pass * 4 + k < valid ? pbuf[(pass * 4 + k) * kG + head] : -INFINITY;
-    __syncwarp();
+        if (pass * 4 + k >= valid) lg[pass] = -INFINITY;
     // online softmax for this lane's head (lanes k = 0..3 share it)
     float pm = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
     pm = fmaxf(pm, __shfl_xor_sync(full, pm, 8));
     pm = fmaxf(pm, __shfl_xor_sync(full, pm, 16));
     const float m_new = fmaxf(st.m, pm);
-    const float alpha = fast_exp2(st.m - m_new);   // st.m = -inf on the first page -> 0
+    // no kept token yet (every token so far dropped): any finite shift works
+    const float m_ref = m_new == -INFINITY ? 0.f : m_new;
+    const float alpha = fast_exp2(st.m - m_ref);   // st.m = -inf on the first page -> 0
     st.m = m_new;
     const __half* vs = (const __half*)(pg + 2 * kP);
     float wv[4];   // vscale * sc of this lane's tokens
@@ -654,13 +761,13 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
     float psum = 0.f;
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
-        const float pv = fast_exp2(lg[pass] - m_new);
+        const float pv = fast_exp2(lg[pass] - m_ref);   // -inf (dropped, past the end) -> 0
         psum += pv;
         const int t = pass * 4 + k;
-        if (s < 4) pbuf[t * kG + head] = pv * wv[pass];
+        if (!(s & 1)) pbuf[t * kG + head] = pv * wv[pass];
     }
     st.l = st.l * alpha + psum;
-    if (lane < 4) pbuf[16 * kG + head] = alpha_acc;
+    if (lane < 8 && !(s & 1)) pbuf[16 * kG + head] = alpha_acc;
     __syncwarp();
 
     page_values<kG>(pg, tier, pbuf, lane, alpha_acc, st);
@@ -671,35 +778,10 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
 // Several decode query tokens per sequence (speculative or chunked decode):
 // a launch takes a pair of them, i.e. 8 query heads per kv head, so one page
 // stream serves both and the tensor-core tile's 8 columns are all used.  The
-// shared memory of the query-folded table holds, instead, the pair's query
-// rows (4 arrays of (q[2j], q[2j+1]) for heads 2a, 2a+1, at byte 1024 a +
-// (144 s ^ 16 i) for leaf j = 8s + i) and the warps' weight buffers; every
-// tier's leaves read (cos, sin) from the T1 leaf table, whose grid holds the
-// others (T2 code c is T1 code 16c, T3 code c is T1 code 32c).
+// pair's query rows sit in shared memory (Layout<2>: 4 arrays of (q[2j],
+// q[2j+1]) for heads 2a, 2a+1, at byte 1024 a + (144 s ^ 16 i) for leaf
+// j = 8s + i); every tier's leaves read (cos, sin) from the T1 leaf rows.
 constexpr int kGQ2 = 2 * kG;                          // heads per unit
-constexpr int kMqQOff = kFoldOff;                      // 4 KB of query rows
-constexpr int kMqPbufFloats = 16 * kGQ2 + 2 * kGQ2;    // weights; alpha; valid counts
-constexpr int kMqPbufOff = kMqQOff + 4 * 1024;
-static_assert(kMqPbufOff + kWarps * kMqPbufFloats * 4 <= kFoldOff + kFoldBytes, "pair buffers");
-static_assert((2 * kWarps * kGQ2 + kWarps * kGQ2 * kD) * 4 <= kWarps * kStages * kStageBytes, "pair merge scratch");
-
-// Offsets of one subtree block's 8 leaf codes (into the T1 leaf table) and 8
-// upper codes (into the tier's upper table).
-template <int T>
-__device__ __forceinline__ void block_offsets_mq(const uint8_t* codes, int blk, uint32_t base_rep,
-                                                 const uint32_t (&fl)[8], uint32_t (&lo)[8], uint32_t (&uo)[8])
-{
-    block_offsets<T>(codes, blk, base_rep, fl, lo, uo);
-    if (T == 2) {
-        const uint32_t w = *(const uint32_t*)(codes + blk * 8);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) lo[j] = (((w >> (4 * j)) & 15u) << 12) | base_rep;
-    } else if (T == 3) {
-        const uint32_t lf = *(const uint16_t*)(codes + kP * 32 + blk * 2) | ((uint32_t)codes[kP * 48 + blk] << 16);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) lo[j] = (((lf >> (3 * j)) & 7u) << 13) | base_rep;
-    }
-}
 
 // One subtree block for the 8 heads of a query pair, top down from its
 // weight v: per head, (q[2j], q[2j+1]) . (w cos phi, w sin phi) summed in
@@ -733,7 +815,7 @@ __device__ __forceinline__ void subtree_mq(float v, const uint32_t (&lo)[8], con
         const float2 kk = make_float2(wl[j] * f.x, wl[j] * f.y);
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
-            const float4 qv = *(const float4*)(smem + kMqQOff + 1024 * a + fl[j]);   // heads 2a, 2a+1
+            const float4 qv = *(const float4*)(smem + Layout<2>::kQ + 1024 * a + fl[j]);   // heads 2a, 2a+1
             const float2 qa = make_float2(qv.x, qv.y), qb = make_float2(qv.z, qv.w);
             acc2[2 * a] = (first && j == 0) ? __fmul2_rn(qa, kk) : __ffma2_rn(qa, kk, acc2[2 * a]);
             acc2[2 * a + 1] = (first && j == 0) ? __fmul2_rn(qb, kk) : __ffma2_rn(qb, kk, acc2[2 * a + 1]);
@@ -766,7 +848,7 @@ __device__ __forceinline__ void page_logits_mq(const uint8_t* pg, const uint8_t*
     for (int pass = 0; pass < 2; ++pass) {
         const int t = pass * 8 + k8;
         uint32_t lo[8], uo[8];
-        block_offsets_mq<T>(codes, t * 8 + sA, rep, flA, lo, uo);
+        block_offsets<T>(codes, t * 8 + sA, rep, lo, uo);
         const uint32_t topB = block_top<T>(codes, t * 8 + sB, rep);
         const uint32_t top2 = (a_right ? topB : uo[7]) | ((a_right ? uo[7] : topB) << 16);
         const uint32_t w4 = __shfl_sync(full, top2, base + (q >> 1));
@@ -775,14 +857,15 @@ __device__ __forceinline__ void page_logits_mq(const uint8_t* pg, const uint8_t*
         const uint32_t o4 = (w4 >> (16 * (q & 1))) & 0xffffu;
         const uint32_t o5 = (w5 >> (16 * (q >> 1))) & 0xffffu;
         const uint32_t o6 = w6 & 0xffffu;
-        float v = __half2float(((const __half*)pg)[t]) * kLogitScale;
+        const uint32_t rb = ((const uint16_t*)pg)[t];   // the sign bit is the token's drop flag
+        float v = __half2float(__ushort_as_half((unsigned short)(rb & 0x7fffu))) * kLogitScale;
         v *= *(const float*)(lut_up + o6 + side6);
         v *= *(const float*)(lut_up + o5 + side5);
         const float2 f4 = *(const float2*)(lut_up + o4);
         const float vA = v * (a_right ? f4.y : f4.x), vB = v * (a_right ? f4.x : f4.y);
         float2 acc2[kGQ2];
         subtree_mq<T>(vA, lo, uo, smem, lut_up, flA, acc2, true);
-        block_offsets_mq<T>(codes, t * 8 + sB, rep, flB, lo, uo);
+        block_offsets<T>(codes, t * 8 + sB, rep, lo, uo);
         subtree_mq<T>(vB, lo, uo, smem, lut_up, flB, acc2, false);
         float acc[kGQ2];
 #pragma unroll
@@ -797,7 +880,8 @@ __device__ __forceinline__ void page_logits_mq(const uint8_t* pg, const uint8_t*
         float y[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) y[h] = (b0 ? x[2 + h] : x[h]) + __shfl_xor_sync(full, b0 ? x[h] : x[2 + h], 1);
-        *(float2*)(pbuf + t * kGQ2 + 2 * q) = make_float2(y[0], y[1]);
+        *(float2*)(pbuf + t * kGQ2 + 2 * q) = (rb & 0x8000u) ? make_float2(-INFINITY, -INFINITY)
+                                                            : make_float2(y[0], y[1]);
     }
 }
 
@@ -875,49 +959,59 @@ __device__ __forceinline__ int64_t out_row(const DecodeParams& p, int b, int g, 
 // ------------------------------------------------------------ decode --
 // NQ = 1: one query token (4 heads per unit); NQ = 2: a pair (8 heads).
 template <int NQ>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
+__global__ void __launch_bounds__(Layout<NQ>::kWarps * 32, 1) decode_kernel(DecodeParams p)
 {
-    constexpr int GQ = NQ == 1 ? kG : kGQ2;   // heads per unit
+    using L = Layout<NQ>;
+    constexpr int kWarps = L::kWarps, kThreads = kWarps * 32, kS = L::kStages;
+    constexpr int GQ = L::kHeads;   // heads per unit
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const unsigned full = 0xffffffffu;
 
+    // Zero point of the layout: shared address 0 for one query (absolute
+    // offsets, the dynamic block must start below the first region), the
+    // dynamic block for a pair.
+    const uint32_t sbase = smem_u32(smem);
+    if constexpr (NQ == 1) {
+        if (sbase > Layout<1>::kUpT2) {   // cannot happen with <= 8 KB of reserved shared memory
+            if (tid == 0) report(p.status, SPHKV_ERR_DEVICE);
+            return;
+        }
+    }
+    uint8_t* const Z = NQ == 1 ? smem - sbase : smem;
+    const uint32_t zs = NQ == 1 ? 0u : sbase;
+
     // cos/sin tables: leaf grid c*2pi/2^b_leaf, upper grid c*(pi/2)/(2^b_up-1)
-    for (int e = tid; e < 2 * 256 + 64 + 16 + 16; e += kThreads) {
+    for (int e = tid; e < 2 * 256 + 64 + 16; e += kThreads) {
         double a;   // angle / pi
-        int off, reps = 16;
+        uint32_t off;
         if (e < 512) {   // T1 row e/2: leaf half, upper half
             const int code = e >> 1, upper = e & 1;
             a = upper ? 0.5 * code / 255 : 2.0 * code / 256;
-            off = kLutT1 + code * 256 + upper * 128;
+            off = L::kT1 + code * 256 + upper * 128;
         } else if (e < 576) {
             a = 0.5 * (e - 512) / 63;
-            off = kLutT2 + (e - 512) * 128;
-        } else if (e < 592) {
-            a = 0.5 * (e - 576) / 15;
-            off = kLutT3 + (e - 576) * 128;
+            off = L::kUpT2 + (e - 512) * 128;
         } else {
-            a = 2.0 * (e - 592) / 16;
-            off = kLeafT2 + (e - 592) * 8;
-            reps = 1;
+            a = 0.5 * (e - 576) / 15;
+            off = L::kUpT3 + (e - 576) * 128;
         }
         double sn, cs;
         sincospi(a, &sn, &cs);
         const float2 v = make_float2((float)cs, (float)sn);
-        for (int r = 0; r < reps; ++r) ((float2*)(smem + off))[r] = v;
+        for (int r = 0; r < 16; ++r) ((float2*)(Z + off))[r] = v;
     }
-    // per-lane offsets of leaf i of subtree s = lane & 7 in the folded table
-    // and the T1 query arrays
+    // pairs: per-lane offsets of leaf i of subtree 2 (lane & 3) + ((lane >> 2)
+    // & 1) in the query arrays
     uint32_t fl[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) fl[i] = (144u * (uint32_t)(2 * (lane & 3) + ((lane >> 2) & 1))) ^ (16u * i);
-    uint8_t* stage = smem + kStageOff + w * kStages * kStageBytes;
-    float* pbuf = NQ == 1 ? (float*)(smem + kPbufOff) + w * kPbufFloats
-                          : (float*)(smem + kMqPbufOff) + w * kMqPbufFloats;
-    const uint32_t bar0 = smem_u32(smem + kBarOff + w * kStages * 8);
+    uint8_t* stage = Z + L::kStage + w * kS * kStageBytes;
+    float* pbuf = (float*)(Z + L::kPbuf) + w * L::kPbufFloats;
+    const uint32_t bar0 = zs + L::kBar + w * kS * 8;
     if (lane == 0) {
-        mbar_init(bar0, 1);
-        mbar_init(bar0 + 8, 1);
+#pragma unroll
+        for (int i = 0; i < kS; ++i) mbar_init(bar0 + 8 * i, 1);
         fence_barrier_init();
     }
     __syncthreads();
@@ -928,7 +1022,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
     uint32_t phase = 0;   // bit s = parity to wait for on stage s
     bool failed = false;
 
-    float* ms_m = (float*)(smem + kStageOff);   // merge scratch, aliases the ring
+    float* ms_m = (float*)(Z + L::kStage);   // merge scratch, aliases the rings
     float* ms_l = ms_m + kWarps * GQ;
     float* ms_o = ms_l + kWarps * GQ;
 
@@ -945,11 +1039,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
         const int32_t* ptab = p.page_table + (int64_t)g * p.total_pages + first;
 
         // Split [pa, pe) among the warps by weight.  Warp w first sums slice w
-        // (pages pa + n k / 16 for k = w, w + 1); after the barrier each warp
-        // finds where the running weight crosses W w / 16 and W (w + 1) / 16.
-        // The split depends only on the page table, so results are
-        // reproducible bit for bit.
-        uint32_t* wsum = (uint32_t*)(smem + kSliceOff);
+        // (pages pa + n k / W for k = w, w + 1); after the barrier each warp
+        // finds where the running weight crosses total * w / W and
+        // total * (w + 1) / W.  The split depends only on the page table, so
+        // results are reproducible bit for bit.
+        uint32_t* wsum = (uint32_t*)(Z + L::kSlice);
         const int32_t n_seg = pe - pa;
         auto slice_start = [&](int k) -> int32_t { return pa + (int32_t)(((int64_t)n_seg * k) / kWarps); };
         {
@@ -958,26 +1052,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
             sum = __reduce_add_sync(full, sum);
             if (lane == 0) wsum[w] = sum;
         }
+        // One query: this lane's query slice in registers, q[16s .. 16s+15] of
+        // the 4 heads times the logit scale, in the lane's slot order (see
+        // page_logits), and the unit's query-folded T2/T3 leaf table (the
+        // previous segment ended with a barrier, so no warp still reads it).
+        float2 qp[kG][8];
         if constexpr (NQ == 1) {
-            // query-folded leaf table for this unit (the previous segment ended
-            // with a barrier, so no warp still reads the old one)
-            for (int e = tid; e < 16 * kLeaves; e += kThreads) {
-                const int code = e >> 6, j = e & 63;
-                const float2 cs = *(const float2*)(smem + kLeafT2 + code * 8);
-                float v[kG];
-    #pragma unroll
-                for (int h = 0; h < kG; ++h) {
-                    const float* qh = p.q + out_row(p, b, g, h) * kD;
-                    v[h] = fmaf(qh[2 * j + 1], cs.y, qh[2 * j] * cs.x);
+            const int s = lane & 7, b2 = (s >> 2) & 1, b1 = (s >> 1) & 1;
+#pragma unroll
+            for (int i = 0; i < kG; ++i) {
+                const int h = (((i >> 1) ^ b2) << 1) | ((i & 1) ^ b1);
+                const float4* src = (const float4*)(p.q + out_row(p, b, g, h) * kD + 16 * s);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 v = src[k];
+                    qp[i][2 * k] = make_float2(v.x * kLogitScale, v.y * kLogitScale);
+                    qp[i][2 * k + 1] = make_float2(v.z * kLogitScale, v.w * kLogitScale);
                 }
-                const uint32_t off = ((uint32_t)code << 10) + 128u * (j >> 3) + 16u * ((j & 7) ^ (j >> 3));
-                *(float4*)(smem + kFoldOff + off) = make_float4(v[0], v[1], v[2], v[3]);
             }
-            for (int e = tid; e < 2 * kLeaves; e += kThreads) {   // q for T1 leaves
-                const int half = e >= kLeaves, j = e & 63, sj = j >> 3, ij = j & 7;
-                const float* q0 = p.q + out_row(p, b, g, 2 * half) * kD + 2 * j;
-                const float* q1 = q0 + kD;
-                *(float4*)(smem + kQOff + 1024 * half + ((144 * sj) ^ (16 * ij))) = make_float4(q0[0], q0[1], q1[0], q1[1]);
+            for (int e = tid; e < 16 * kLeaves; e += kThreads) {
+                const int code = e >> 6, j = e & 63, sj = j >> 3, ij = j & 7;
+                const int c2 = (sj >> 2) & 1, c1 = (sj >> 1) & 1;   // slot order of the lanes owning subtree sj
+                const float2 cs = *(const float2*)(Z + L::kT1 + 16 * code * 256);   // T2 code c = T1 code 16c
+                float v[kG];
+#pragma unroll
+                for (int k = 0; k < kG; ++k) {
+                    const int h = (((k >> 1) ^ c2) << 1) | ((k & 1) ^ c1);
+                    const float* qh = p.q + out_row(p, b, g, h) * kD;
+                    v[k] = fmaf(qh[2 * j + 1], cs.y, qh[2 * j] * cs.x) * kLogitScale;
+                }
+                *(float4*)(Z + L::kFold + ((uint32_t)code << 11) + 144 * sj + 16 * ij) =
+                    make_float4(v[0], v[1], v[2], v[3]);
             }
         } else {   // the pair's query rows (the previous segment ended with a barrier)
             for (int e = tid; e < 4 * kLeaves; e += kThreads) {
@@ -991,7 +1096,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
                     v[2 * hp] = live ? qh[0] : 0.f;
                     v[2 * hp + 1] = live ? qh[1] : 0.f;
                 }
-                *(float4*)(smem + kMqQOff + 1024 * a + ((144 * sj) ^ (16 * ij))) = make_float4(v[0], v[1], v[2], v[3]);
+                *(float4*)(Z + L::kQ + 1024 * a + ((144 * sj) ^ (16 * ij))) = make_float4(v[0], v[1], v[2], v[3]);
             }
         }
         __syncthreads();
@@ -1005,7 +1110,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
                 if (lane >= o) incl += y;
             }
             const int64_t W = __shfl_sync(full, incl, kWarps - 1);
-            // first page whose running weight (itself included) exceeds W k / 16
+            // first page whose running weight (itself included) exceeds W k / kWarps
             auto boundary = [&](int k) -> int32_t {
                 if (k == 0) return pa;
                 if (k == kWarps) return pe;
@@ -1083,23 +1188,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
                 bulk_g2s(smem_u32(stage + stg * kStageBytes), page_src(e), bytes, bar0 + 8 * stg);
             }
         };
+        // Pages in flight: slot i of (lpq, eq, hq) is the page i places ahead
+        // of the one being computed, staged in ring stage (cur + i) % kS.
         Cursor cur_c{0, 0, 0u};
         refill(cur_c);
-        int32_t lp_cur = 0, e_cur = 0, lp_nxt = 0, e_nxt = 0;
-        bool have_cur = advance(cur_c, lp_cur, e_cur);
+        int32_t lpq[kS], eq[kS];
+        bool hq[kS];
+#pragma unroll
+        for (int i = 0; i < kS; ++i) {
+            lpq[i] = 0;
+            eq[i] = 0;
+            hq[i] = false;
+        }
+        hq[0] = advance(cur_c, lpq[0], eq[0]);
+#pragma unroll
+        for (int i = 1; i < kS - 1; ++i) hq[i] = hq[i - 1] && advance(cur_c, lpq[i], eq[i]);
         int cur = 0;
 #ifdef SPHKV_TEST_HOOKS
-        const bool skip_first = p.test_skip_copy && blockIdx.x == 0 && w == 0 && x == lo;
+        // warp 0 of CTA 0 alone skips its first copy and waits with a short limit
+        const bool hooked = p.test_skip_copy && blockIdx.x == 0 && w == 0;
+        const bool skip_first = hooked && x == lo;
 #else
         constexpr bool skip_first = false;
 #endif
-        if (have_cur && !skip_first) issue(0, e_cur);
-        while (have_cur) {
-            const bool have_nxt = advance(cur_c, lp_nxt, e_nxt);
-            if (have_nxt) issue(cur ^ 1, e_nxt);
+#pragma unroll
+        for (int i = 0; i < kS - 1; ++i)
+            if (hq[i] && !(i == 0 && skip_first)) issue(i, eq[i]);
+        while (hq[0]) {
+            // the page kS - 1 ahead goes into the stage the previous page used
+            hq[kS - 1] = hq[kS - 2] && advance(cur_c, lpq[kS - 1], eq[kS - 1]);
+            if (hq[kS - 1]) issue(cur == 0 ? kS - 1 : cur - 1, eq[kS - 1]);
 #ifdef SPHKV_TEST_HOOKS
-            const bool ok = p.test_skip_copy ? mbar_wait<(1L << 12)>(bar0 + 8 * cur, (phase >> cur) & 1)
-                                             : mbar_wait(bar0 + 8 * cur, (phase >> cur) & 1);
+            const bool ok = hooked ? mbar_wait<(1L << 12)>(bar0 + 8 * cur, (phase >> cur) & 1)
+                                   : mbar_wait(bar0 + 8 * cur, (phase >> cur) & 1);
 #else
             const bool ok = mbar_wait(bar0 + 8 * cur, (phase >> cur) & 1);
 #endif
@@ -1107,40 +1228,54 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(DecodeParams p)
             if (!ok) {
                 if (lane == 0) report(p.status, SPHKV_ERR_TIMEOUT);
                 failed = true;
-                if (have_nxt) {   // drain the copy still in flight, again bounded
-                    mbar_wait(bar0 + 8 * (cur ^ 1), (phase >> (cur ^ 1)) & 1);
-                    phase ^= 1u << (cur ^ 1);
+                // drain the copies still in flight, again bounded
+#pragma unroll
+                for (int i = 1; i < kS; ++i) {
+                    if (!hq[i]) break;
+                    const int sg = (cur + i) % kS;
+                    mbar_wait(bar0 + 8 * sg, (phase >> sg) & 1);
+                    phase ^= 1u << sg;
                 }
                 break;
             }
             const uint8_t* pg = stage + cur * kStageBytes;
-            const int t = entry_tier(e_cur);
+            const int t = entry_tier(eq[0]);
             if constexpr (NQ == 1) {
-                const int valid = min(kP, len - lp_cur * kP);
-                process_page(pg, t, valid, smem, pbuf, lane, fl, st);
+                const int valid = min(kP, len - lpq[0] * kP);
+                process_page(pg, t, valid, pbuf, lane, qp, st);
             } else {
-                const int v0 = max(0, min(kP, len - lp_cur * kP)), v1 = max(0, min(kP, len2 - lp_cur * kP));
+                const int v0 = max(0, min(kP, len - lpq[0] * kP)), v1 = max(0, min(kP, len2 - lpq[0] * kP));
                 process_page_mq(pg, t, v0, v1, smem, pbuf, lane, fl, st);
             }
-            cur ^= 1;
-            lp_cur = lp_nxt;
-            e_cur = e_nxt;
-            have_cur = have_nxt;
+#pragma unroll
+            for (int i = 0; i < kS - 1; ++i) {
+                lpq[i] = lpq[i + 1];
+                eq[i] = eq[i + 1];
+                hq[i] = hq[i + 1];
+            }
+            hq[kS - 1] = false;
+            cur = cur + 1 == kS ? 0 : cur + 1;
         }
 
-        // ---- CTA merge of the 16 warps' (m, l, o) for this segment
-        float lt = st.l;   // lanes s and s+4 duplicate: sum over k only
+        // ---- CTA merge of the warps' (m, l, o) for this segment
+        float lt = st.l;   // lanes with the same head duplicate: sum over k only
         lt += __shfl_xor_sync(full, lt, 8);
         lt += __shfl_xor_sync(full, lt, 16);
+        if constexpr (NQ == 1) {   // hi and lo weight columns (lanes c, c ^ 2) add up
+#pragma unroll
+            for (int m = 0; m < 8; ++m)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) st.acc[m][i] += __shfl_xor_sync(full, st.acc[m][i], 2);
+        }
         // every warp is done with its ring; a timed-out copy in any warp ends
         // the whole CTA after this segment (every warp leaves the loop together)
         failed = __syncthreads_or(failed);
         {
             const int s = lane & 7;
-            // the softmax head of lane (k, s): (s & 1) * 2 + ((s >> 1) & 1) for
-            // one query (lanes s, s + 4 alike), s for a pair
-            const int head = NQ == 1 ? (s & 1) * 2 + ((s >> 1) & 1) : s;
-            if (lane < GQ) {
+            // the softmax head of lane (k, s): (s >> 2) * 2 + ((s >> 1) & 1) for
+            // one query (lanes s, s ^ 1 alike), s for a pair
+            const int head = NQ == 1 ? (s >> 2) * 2 + ((s >> 1) & 1) : s;
+            if (NQ == 1 ? (lane < 8 && !(s & 1)) : lane < GQ) {
                 ms_m[w * GQ + head] = st.m;
                 ms_l[w * GQ + head] = lt;
             }
@@ -1251,8 +1386,8 @@ void launch_decode(const DecodeParams& p, cudaStream_t s)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(p.n_cta);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.blockDim = dim3(Layout<NQ>::kWarps * 32);
+    cfg.dynamicSmemBytes = Layout<NQ>::kSmemBytes;
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
@@ -1359,11 +1494,11 @@ sphkv_status ensure_smem(const char* fn)
         return SPHKV_ERR_DEVICE;
     }
     if (attr_dev != dev) {
-        if (cudaFuncSetAttribute(decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-                cudaSuccess) {
-            sphkv_set_error("%s: cannot reserve %d bytes of shared memory", fn, kSmemBytes);
+        if (cudaFuncSetAttribute(decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Layout<1>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Layout<2>::kSmemBytes) != cudaSuccess) {
+            sphkv_set_error("%s: cannot reserve %d bytes of shared memory", fn, Layout<2>::kSmemBytes);
             return SPHKV_ERR_DEVICE;
         }
         attr_dev = dev;
@@ -1479,9 +1614,6 @@ extern "C" sphkv_status sphkv_decode_attention_mq(const sphkv_cache* c, int32_t 
 namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;   // 4 MiB per device
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kMaxDevices] = {};
 }  // namespace
 
 extern "C" sphkv_status sphkv_decode_attention_noalloc(const sphkv_cache* c, int32_t H_q, const float* q,
@@ -1500,28 +1632,17 @@ extern "C" sphkv_status sphkv_decode_attention_noalloc(const sphkv_cache* c, int
                         fn, need, kNoAllocScratchBytes);
         return SPHKV_ERR_ARG;
     }
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-        sphkv_set_error("%s: no usable current device", fn);
-        return SPHKV_ERR_DEVICE;
-    }
+    // The device address of the static array, looked up with the caller's
+    // device current (a host-side symbol is not a device address).  It is
+    // looked up on every call, which costs no allocation and stays right after
+    // a device reset or a context switch; the first call on a device also
+    // loads the module there, so make that first call before any stream
+    // capture.
     void* scratch = nullptr;
-    {
-        // First call on each device: look up the device address of the static
-        // array with that device current (a host-side symbol is not a device
-        // address).  This first call should come before any stream capture.
-        std::lock_guard<std::mutex> lock(g_noalloc_mu);
-        if (!g_noalloc_addr[dev]) {
-            void* a = nullptr;
-            const cudaError_t e = cudaGetSymbolAddress(&a, g_noalloc_scratch);
-            if (e != cudaSuccess || !a) {
-                sphkv_set_error("%s: cudaGetSymbolAddress failed: %s", fn, cudaGetErrorString(e));
-                return SPHKV_ERR_DEVICE;
-            }
-            if ((st = ensure_smem(fn)) != SPHKV_OK) return st;
-            g_noalloc_addr[dev] = a;
-        }
-        scratch = g_noalloc_addr[dev];
+    const cudaError_t e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
+    if (e != cudaSuccess || !scratch) {
+        sphkv_set_error("%s: cudaGetSymbolAddress failed: %s", fn, cudaGetErrorString(e));
+        return SPHKV_ERR_DEVICE;
     }
     if ((st = ensure_smem(fn)) != SPHKV_OK) return st;
     p.unit_start = (int32_t*)scratch;

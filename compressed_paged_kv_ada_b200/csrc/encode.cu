@@ -77,6 +77,10 @@ __device__ inline uint32_t block_up(const uint8_t* up, int s, int j)
 }
 
 template <int T>
+__device__ void pack_token(uint8_t* page, int slot, const uint8_t* sleaf, const uint8_t* sup, const int8_t* vq,
+                           int lane);
+
+template <int T>
 __device__ void encode_token(const EncParams& p, int64_t i, int g, uint8_t* page, int slot,
                              uint8_t* sleaf, uint8_t* sup, int lane)
 {
@@ -126,6 +130,24 @@ __device__ void encode_token(const EncParams& p, int64_t i, int g, uint8_t* page
 #pragma unroll
     for (int c = 0; c < 4; ++c) vq[4 * lane + c] = (int8_t)q[c];
     __syncwarp();
+    pack_token<T>(page, slot, sleaf, sup, vq, lane);
+    if (lane == 0) {
+        __half r16 = __double2half(sqrt(ss));
+        ((__half*)page)[slot] = r16;
+        ((__half*)(page + 2 * kP))[slot] = s16;
+        if (__hisinf(r16) || __hisinf(s16)) report(p.status, SPHKV_ERR_RANGE);
+    }
+}
+
+// Write one token's codes (leaf[64], upper[63] in level order) and value
+// codes vq[128] (by channel) into slot `slot` of a tier-T page, in the
+// format of include/sphkv.h; the radius and scale are written by the caller.
+// The whole warp takes part.
+template <int T>
+__device__ void pack_token(uint8_t* page, int slot, const uint8_t* sleaf, const uint8_t* sup, const int8_t* vq,
+                           int lane)
+{
+    constexpr TierFmt F = Tier<T>::f;
     // code blocks: 8 per token; lane l writes 32-bit word l of the token's blocks
     uint8_t* codes = page + F.off_codes;
     if (T == 1) {   // block s = 16 bytes: 8 leaf codes then 8 upper codes
@@ -189,12 +211,6 @@ __device__ void encode_token(const EncParams& p, int64_t i, int g, uint8_t* page
         const int g = lane >> 1, i = slot >> 1;
         *(uint32_t*)(vsec + i * 128 + 16 * (g ^ ((2 * i) & 6)) + 8 * (slot & 1) + 4 * (lane & 1)) = w;
     }
-    if (lane == 0) {
-        __half r16 = __double2half(sqrt(ss));
-        ((__half*)page)[slot] = r16;
-        ((__half*)(page + 2 * kP))[slot] = s16;
-        if (__hisinf(r16) || __hisinf(s16)) report(p.status, SPHKV_ERR_RANGE);
-    }
 }
 
 __global__ void __launch_bounds__(kEncWarps * 32) encode_kernel(EncParams p)
@@ -231,10 +247,238 @@ __global__ void __launch_bounds__(kEncWarps * 32) encode_kernel(EncParams p)
     else encode_token<3>(p, i, g, page, slot, s_leaf[wib], s_up[wib], lane);
 }
 
+// ------------------------------------------------------------ migrate --
+// After RDR runs again (sphkv_rdr_rerun) a page may move to a coarser tier;
+// its tokens are transcoded from their codes alone.  The rule (this library's
+// reading; the pages give none): each angle goes to the nearest point of the
+// coarser grid, computed exactly on the code integers with ties to even; the
+// radius and its drop flag are kept; the values are decoded (code * scale,
+// exact in fp64) and quantised again with the encoder's rule for the new
+// width.  A token whose tier does not change moves unchanged.
+
+struct MigParams {
+    int B, H_kv;
+    int64_t total_pages;
+    const int32_t* page_offsets;
+    const int32_t* seq_lens;
+    const int32_t* old_table;
+    const uint8_t* old_pool[4];
+    int64_t old_pages[4];
+    const int32_t* new_table;
+    uint8_t* new_pool[4];
+    int64_t new_pages[4];
+    int32_t* status;
+};
+
+// Round-half-even of num / den (num >= 0, den > 0).
+__device__ inline int64_t div_rne(int64_t num, int64_t den)
+{
+    int64_t q = num / den;
+    const int64_t r = num - q * den;
+    if (2 * r > den || (2 * r == den && (q & 1))) ++q;
+    return q;
+}
+
+// Nearest point of the coarser periodic leaf grid (2^b_to points).
+__device__ inline int leaf_to(int c, int b_from, int b_to)
+{
+    return (int)(div_rne((int64_t)c << b_to, (int64_t)1 << b_from) & (((int64_t)1 << b_to) - 1));
+}
+
+// Nearest point of the coarser end-inclusive upper grid (2^b_to - 1 steps).
+__device__ inline int upper_to(int c, int b_from, int b_to)
+{
+    return (int)div_rne((int64_t)c * ((1 << b_to) - 1), (int64_t)(1 << b_from) - 1);
+}
+
+// Read slot `slot` of a tier-T page into leaf[64], up[63] (level order) and
+// vq[128] (by channel); the whole warp takes part.
+template <int T>
+__device__ void unpack_token(const uint8_t* page, int slot, uint8_t* sleaf, uint8_t* sup, int8_t* vq, int lane)
+{
+    constexpr TierFmt F = Tier<T>::f;
+    const uint8_t* codes = page + F.off_codes;
+    if (lane < 8) {   // block s = lane
+        const int s = lane, blk = slot * 8 + s;
+        uint32_t L[8], U[8];
+        if (T == 1) {
+            const uint8_t* b = codes + blk * 16;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                L[j] = b[j];
+                U[j] = b[8 + j];
+            }
+        } else if (T == 2) {
+            const uint64_t a = *(const uint64_t*)(codes + blk * 8);
+            const uint64_t uf = (a >> 32) | ((uint64_t)*(const uint16_t*)(codes + kP * 64 + blk * 2) << 32);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                L[j] = (uint32_t)(a >> (4 * j)) & 15u;
+                U[j] = (uint32_t)(uf >> (6 * j)) & 63u;
+            }
+        } else {
+            const uint32_t u = *(const uint32_t*)(codes + blk * 4);
+            const uint32_t lf = *(const uint16_t*)(codes + kP * 32 + blk * 2) | ((uint32_t)codes[kP * 48 + blk] << 16);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                U[j] = (u >> (4 * j)) & 15u;
+                L[j] = (lf >> (3 * j)) & 7u;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sleaf[8 * s + j] = (uint8_t)L[j];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sup[4 * s + j] = (uint8_t)U[j];
+        sup[32 + 2 * s] = (uint8_t)U[4];
+        sup[32 + 2 * s + 1] = (uint8_t)U[5];
+        sup[48 + s] = (uint8_t)U[6];
+        if (s < 7) sup[56 + s] = (uint8_t)U[7];
+    }
+    const uint8_t* vsec = page + F.off_v;
+    if (F.v_bits == 8) {
+        const int g = lane >> 2;
+        const uint32_t w = *(const uint32_t*)(vsec + slot * 128 + 16 * (g ^ (slot & 6)) + 4 * (lane & 3));
+#pragma unroll
+        for (int b = 0; b < 4; ++b) vq[v_channel_at(4 * lane + b)] = (int8_t)(w >> (8 * b));
+    } else if (lane < 16) {
+        const int g = lane >> 1, i = slot >> 1;
+        const uint32_t w =
+            *(const uint32_t*)(vsec + i * 128 + 16 * (g ^ ((2 * i) & 6)) + 8 * (slot & 1) + 4 * (lane & 1));
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            int x = (int)((w >> (4 * b)) & 15u);
+            vq[v_channel_at(8 * lane + b)] = (int8_t)(x >= 8 ? x - 16 : x);   // two's complement nibble
+        }
+    }
+}
+
+template <int TF>
+__device__ void unpack_any(int tf, const uint8_t* page, int slot, uint8_t* sleaf, uint8_t* sup, int8_t* vq, int lane)
+{
+    if (tf == 1) unpack_token<1>(page, slot, sleaf, sup, vq, lane);
+    else if (tf == 2) unpack_token<2>(page, slot, sleaf, sup, vq, lane);
+    else unpack_token<3>(page, slot, sleaf, sup, vq, lane);
+}
+
+__device__ inline int bits_leaf(int t) { return t == 1 ? 8 : t == 2 ? 4 : 3; }
+__device__ inline int bits_up(int t) { return t == 1 ? 8 : t == 2 ? 6 : 4; }
+
+__global__ void __launch_bounds__(kEncWarps * 32) migrate_kernel(MigParams p)
+{
+    __shared__ uint8_t s_leaf[kEncWarps][kLeaves];
+    __shared__ uint8_t s_up[kEncWarps][kUpper + 1];
+    __shared__ int8_t s_vq[kEncWarps][kD];
+    const unsigned full = 0xffffffffu;
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int64_t per_head = p.total_pages * kP;
+    const int64_t wg = (int64_t)blockIdx.x * kEncWarps + wib;   // (kv head, logical page, slot)
+    if (wg >= per_head * p.H_kv) return;
+    const int g = (int)(wg / per_head);
+    const int64_t lp = (wg % per_head) / kP;
+    const int slot = (int)(wg % kP);
+    int lo = 0, hi = p.B - 1;   // sequence owning logical page lp
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.page_offsets[mid] <= lp) lo = mid;
+        else hi = mid - 1;
+    }
+    if (lp >= p.page_offsets[lo + 1]) return;
+    if ((lp - p.page_offsets[lo]) * kP + slot >= p.seq_lens[lo]) return;   // no token in this slot
+    const int32_t eo = p.old_table[(int64_t)g * p.total_pages + lp], en = p.new_table[(int64_t)g * p.total_pages + lp];
+    const int to = entry_tier(eo), tn = entry_tier(en);
+    if (tn == 0) return;
+    if (to == 0 || tn < to || entry_page(eo) >= p.old_pages[to] || entry_page(en) >= p.new_pages[tn]) {
+        if (lane == 0) report(p.status, SPHKV_ERR_DATA);   // a page cannot become finer or come back
+        return;
+    }
+    const uint8_t* src = p.old_pool[to] + entry_page(eo) * (int64_t)page_bytes_of(to);
+    uint8_t* dst = p.new_pool[tn] + entry_page(en) * (int64_t)page_bytes_of(tn);
+    uint8_t* sleaf = s_leaf[wib];
+    uint8_t* sup = s_up[wib];
+    int8_t* vq = s_vq[wib];
+    unpack_any<0>(to, src, slot, sleaf, sup, vq, lane);
+    __syncwarp();
+    uint16_t s16 = ((const uint16_t*)(src + 2 * kP))[slot];
+    if (tn != to) {
+        for (int j = lane; j < kLeaves; j += 32) sleaf[j] = (uint8_t)leaf_to(sleaf[j], bits_leaf(to), bits_leaf(tn));
+        for (int j = lane; j < kUpper; j += 32) sup[j] = (uint8_t)upper_to(sup[j], bits_up(to), bits_up(tn));
+        const double sa = (double)__half2float(__ushort_as_half(s16));
+        double v[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) v[c] = __dmul_rn((double)vq[4 * lane + c], sa);
+        double a = fmax(fmax(fabs(v[0]), fabs(v[1])), fmax(fabs(v[2]), fabs(v[3])));
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) a = fmax(a, __shfl_xor_sync(full, a, o));
+        const double Q = tn == 1 ? 127.0 : 7.0;
+        const __half sb = __double2half(__ddiv_rn(a, Q));
+        const double sv = (double)__half2float(sb);
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const double t = sv == 0.0 ? 0.0 : rint(__ddiv_rn(v[c], sv));
+            vq[4 * lane + c] = (int8_t)fmin(fmax(t, -Q), Q);
+        }
+        s16 = __half_as_ushort(sb);
+        if (lane == 0 && __hisinf(sb)) report(p.status, SPHKV_ERR_RANGE);
+    }
+    __syncwarp();
+    if (tn == 1) pack_token<1>(dst, slot, sleaf, sup, vq, lane);
+    else if (tn == 2) pack_token<2>(dst, slot, sleaf, sup, vq, lane);
+    else pack_token<3>(dst, slot, sleaf, sup, vq, lane);
+    if (lane == 0) {
+        ((uint16_t*)dst)[slot] = ((const uint16_t*)src)[slot];   // radius and drop flag unchanged
+        ((uint16_t*)(dst + 2 * kP))[slot] = s16;
+    }
+}
+
 }  // namespace
 }  // namespace sphkv
 
 using namespace sphkv;
+
+extern "C" sphkv_status sphkv_migrate(const sphkv_cache* from, const sphkv_cache* to, int32_t* status_dev,
+                                      void* stream)
+{
+    const char* fn = "sphkv_migrate";
+    if (!from || !to) {
+        sphkv_set_error("%s: null argument", fn);
+        return SPHKV_ERR_ARG;
+    }
+    if (from->B <= 0 || from->H_kv <= 0 || from->total_pages < 0 || !from->page_offsets || !from->seq_lens ||
+        !from->page_table || !to->page_table || from->B != to->B || from->H_kv != to->H_kv ||
+        from->total_pages != to->total_pages) {
+        sphkv_set_error("%s: the two cache descriptors must describe the same sequences and pages", fn);
+        return SPHKV_ERR_ARG;
+    }
+    if ((int64_t)from->H_kv * from->total_pages * kP / kEncWarps > 0x7fffffffLL) {
+        sphkv_set_error("%s: cache too large", fn);
+        return SPHKV_ERR_ARG;
+    }
+    MigParams p{};
+    p.B = from->B;
+    p.H_kv = from->H_kv;
+    p.total_pages = from->total_pages;
+    p.page_offsets = from->page_offsets;
+    p.seq_lens = from->seq_lens;
+    p.old_table = from->page_table;
+    p.new_table = to->page_table;
+    for (int t = 1; t <= 3; ++t) {
+        p.old_pool[t] = from->pool[t - 1];
+        p.old_pages[t] = from->pool[t - 1] ? from->pool_pages[t - 1] : 0;
+        p.new_pool[t] = to->pool[t - 1];
+        p.new_pages[t] = to->pool[t - 1] ? to->pool_pages[t - 1] : 0;
+    }
+    p.status = status_dev;
+    const int64_t warps = from->H_kv * from->total_pages * kP;
+    if (warps == 0) return SPHKV_OK;
+    migrate_kernel<<<(unsigned)((warps + kEncWarps - 1) / kEncWarps), kEncWarps * 32, 0, (cudaStream_t)stream>>>(p);
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) {
+        sphkv_set_error("%s: launch failed: %s", fn, cudaGetErrorString(err));
+        return SPHKV_ERR_DEVICE;
+    }
+    return SPHKV_OK;
+}
 
 extern "C" sphkv_status sphkv_encode(const sphkv_cache* c, const void* K, const void* V, int dtype,
                                      const int32_t* tok_seq, const int32_t* tok_pos, int64_t n_tok,

@@ -36,6 +36,7 @@ struct RdrParams {
     int64_t budget;
     int n_sink, n_recent;
     uint8_t* tiers_out;
+    const uint8_t* cap;        // re-run: current tiers, each unit may only get coarser (null: none)
     double* lambda_out;
     int64_t* bytes_out;
     int32_t* status;
@@ -45,14 +46,16 @@ struct RdrParams {
     unsigned int* bar;         // grid barrier counter (zeroed before launch)
     int* abort_flag;
     double* U;                 // [n_units] page utility
-    uint8_t* forced;           // [n_units]
+    uint8_t* forced;           // [n_units]: bit 2 forced, bits 0..1 the finest allowed choice
 };
 
-__device__ inline int choice(double U, const double* eps, const double* R, double lam)
+// argmin over choices first..3 (T1, T2, T3, drop) of U eps + lambda R, ties to
+// the lower index.
+__device__ inline int choice(double U, const double* eps, const double* R, double lam, int first)
 {
-    int best = 0;
-    double bc = __dadd_rn(__dmul_rn(U, eps[0]), __dmul_rn(lam, R[0]));
-    for (int t = 1; t < 4; ++t) {
+    int best = first;
+    double bc = __dadd_rn(__dmul_rn(U, eps[first]), __dmul_rn(lam, R[first]));
+    for (int t = first + 1; t < 4; ++t) {
         double c = __dadd_rn(__dmul_rn(U, eps[t]), __dmul_rn(lam, R[t]));
         if (c < bc) {
             bc = c;
@@ -118,7 +121,8 @@ __global__ void __launch_bounds__(kRdrThreads) rdr_kernel(RdrParams p)
     unsigned gen = 0;
 
     // Page utilities, summed once in slot order (fp64), and the forced flags.
-    // The forced bytes are exact: every forced unit costs a T1 page.
+    // The forced bytes are exact: every forced unit costs the page of the
+    // finest tier it may take (T1 unless a re-run caps it).
     unsigned long long forced_mine = 0;
     for (int64_t u = gtid; u < n_units; u += stride) {
         int32_t pg, np;
@@ -129,9 +133,14 @@ __global__ void __launch_bounds__(kRdrThreads) rdr_kernel(RdrParams p)
         double s = 0.0;
         for (int k = 0; k < kP && pg * kP + k < len; ++k) s = __dadd_rn(s, (double)ut[k]);
         const bool forced = pg < p.n_sink || pg >= np - p.n_recent;
+        int first = 0;   // a re-run may only make a unit coarser
+        if (p.cap) {
+            const int ct = p.cap[e];
+            first = ct == 0 ? 3 : (ct <= 3 ? ct - 1 : 3);
+        }
         p.U[u] = s;
-        p.forced[u] = forced ? 1 : 0;
-        if (forced) forced_mine += (unsigned long long)p.rate[0];
+        p.forced[u] = (uint8_t)((forced ? 4 : 0) | first);
+        if (forced) forced_mine += (unsigned long long)p.rate[first];
     }
     // Block-sum `mine` into acc[slot], then a grid barrier.
     auto commit = [&](unsigned long long mine, int slot) -> bool {
@@ -150,7 +159,10 @@ __global__ void __launch_bounds__(kRdrThreads) rdr_kernel(RdrParams p)
     auto eval = [&](double lam, int slot) -> bool {   // bytes(lam) into acc[slot]
         unsigned long long mine = 0;
         for (int64_t u = gtid; u < n_units; u += stride)
-            mine += (unsigned long long)(p.forced[u] ? p.rate[0] : p.rate[choice(p.U[u], p.eps, p.rate, lam)]);
+        {
+            const int f = p.forced[u], first = f & 3;
+            mine += (unsigned long long)((f & 4) ? p.rate[first] : p.rate[choice(p.U[u], p.eps, p.rate, lam, first)]);
+        }
         return commit(mine, slot);
     };
     auto total = [&](int slot) -> int64_t { return (int64_t)(*(volatile unsigned long long*)(p.acc + slot)); };
@@ -187,7 +199,8 @@ __global__ void __launch_bounds__(kRdrThreads) rdr_kernel(RdrParams p)
         int32_t pg, np;
         int b;
         const int64_t e = unit_entry(p, pages_per_head, u, &pg, &np, &b);
-        const int t = p.forced[u] ? 0 : choice(p.U[u], p.eps, p.rate, hi);
+        const int f = p.forced[u], first = f & 3;
+        const int t = (f & 4) ? first : choice(p.U[u], p.eps, p.rate, hi, first);
         p.tiers_out[e] = (uint8_t)(t == 3 ? 0 : t + 1);
     }
     if (gtid == 0) {
@@ -336,32 +349,58 @@ extern "C" size_t sphkv_rdr_workspace_bytes(int32_t B, int32_t H_kv, int64_t tot
     return rdr_ws_layout(B, H_kv, total_pages, &a, &b, &u, &f);
 }
 
+namespace {
+sphkv_status rdr_launch(const char* fn, bool rerun, const sphkv_cache* c, const float* utility, const double* eps,
+                        int64_t budget_bytes, int32_t n_sink, int32_t n_recent, uint8_t* tiers_out,
+                        double* lambda_out, int64_t* bytes_out, void* workspace, size_t ws_bytes,
+                        int32_t* status_dev, void* stream);
+}
+
 extern "C" sphkv_status sphkv_rdr_assign(const sphkv_cache* c, const float* utility, const double* eps,
                                          int64_t budget_bytes, int32_t n_sink, int32_t n_recent,
                                          uint8_t* tiers_out, double* lambda_out, int64_t* bytes_out,
                                          void* workspace, size_t ws_bytes, int32_t* status_dev,
                                          void* stream)
 {
+    return rdr_launch("sphkv_rdr_assign", false, c, utility, eps, budget_bytes, n_sink, n_recent, tiers_out,
+                      lambda_out, bytes_out, workspace, ws_bytes, status_dev, stream);
+}
+
+extern "C" sphkv_status sphkv_rdr_rerun(const sphkv_cache* c, const float* utility, const double* eps,
+                                        int64_t budget_bytes, int32_t n_sink, int32_t n_recent, uint8_t* tiers_io,
+                                        double* lambda_out, int64_t* bytes_out, void* workspace, size_t ws_bytes,
+                                        int32_t* status_dev, void* stream)
+{
+    return rdr_launch("sphkv_rdr_rerun", true, c, utility, eps, budget_bytes, n_sink, n_recent, tiers_io,
+                      lambda_out, bytes_out, workspace, ws_bytes, status_dev, stream);
+}
+
+namespace {
+sphkv_status rdr_launch(const char* fn, bool rerun, const sphkv_cache* c, const float* utility, const double* eps,
+                        int64_t budget_bytes, int32_t n_sink, int32_t n_recent, uint8_t* tiers_out,
+                        double* lambda_out, int64_t* bytes_out, void* workspace, size_t ws_bytes,
+                        int32_t* status_dev, void* stream)
+{
     if (!c || !utility || !eps || !tiers_out || !lambda_out || !bytes_out || !workspace) {
-        sphkv_set_error("sphkv_rdr_assign: null argument");
+        sphkv_set_error("%s: null argument", fn);
         return SPHKV_ERR_ARG;
     }
     if (c->B <= 0 || c->H_kv <= 0 || !c->page_offsets || !c->seq_lens || c->total_pages < 0) {
-        sphkv_set_error("sphkv_rdr_assign: bad cache descriptor");
+        sphkv_set_error("%s: bad cache descriptor", fn);
         return SPHKV_ERR_ARG;
     }
     if (n_sink < 0 || n_recent < 0 || budget_bytes < 0) {
-        sphkv_set_error("sphkv_rdr_assign: n_sink, n_recent and budget must be >= 0");
+        sphkv_set_error("%s: n_sink, n_recent and budget must be >= 0", fn);
         return SPHKV_ERR_ARG;
     }
     if ((int64_t)c->H_kv * c->total_pages > 0x7fffffffLL) {
-        sphkv_set_error("sphkv_rdr_assign: cache too large for 32-bit page indices");
+        sphkv_set_error("%s: cache too large for 32-bit page indices", fn);
         return SPHKV_ERR_ARG;
     }
     size_t acc_off, bar_off, u_off, f_off;
     const size_t need = rdr_ws_layout(c->B, c->H_kv, c->total_pages, &acc_off, &bar_off, &u_off, &f_off);
     if (ws_bytes < need || ((uintptr_t)workspace & 255)) {
-        sphkv_set_error("sphkv_rdr_assign: workspace must be 256-byte aligned and >= %zu bytes", need);
+        sphkv_set_error("%s: workspace must be 256-byte aligned and >= %zu bytes", fn, need);
         return SPHKV_ERR_ARG;
     }
     RdrParams p{};
@@ -378,6 +417,7 @@ extern "C" sphkv_status sphkv_rdr_assign(const sphkv_cache* c, const float* util
     p.n_sink = n_sink;
     p.n_recent = n_recent;
     p.tiers_out = tiers_out;
+    p.cap = rerun ? tiers_out : nullptr;   // read per unit before the same unit's write
     p.lambda_out = lambda_out;
     p.bytes_out = bytes_out;
     p.status = status_dev;
@@ -390,7 +430,7 @@ extern "C" sphkv_status sphkv_rdr_assign(const sphkv_cache* c, const float* util
     p.forced = ws + f_off;
     cudaStream_t s = (cudaStream_t)stream;
     if (cudaMemsetAsync(ws + acc_off, 0, 512, s) != cudaSuccess) {
-        sphkv_set_error("sphkv_rdr_assign: memset failed");
+        sphkv_set_error("%s: memset failed", fn);
         return SPHKV_ERR_DEVICE;
     }
     seq_scan_kernel<<<1, 1024, 0, s>>>(c->seq_lens, c->page_offsets, c->B, c->total_pages, p.seq_start,
@@ -400,7 +440,7 @@ extern "C" sphkv_status sphkv_rdr_assign(const sphkv_cache* c, const float* util
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rdr_kernel, kRdrThreads, 0);
     if (per_sm < 1 || n_sm < 1) {
-        sphkv_set_error("sphkv_rdr_assign: no cooperative occupancy");
+        sphkv_set_error("%s: no cooperative occupancy", fn);
         return SPHKV_ERR_DEVICE;
     }
     void* args[] = {&p};
@@ -408,11 +448,12 @@ extern "C" sphkv_status sphkv_rdr_assign(const sphkv_cache* c, const float* util
                                                   args, 0, s);
     if (err == cudaSuccess) err = cudaGetLastError();
     if (err != cudaSuccess) {
-        sphkv_set_error("sphkv_rdr_assign: launch failed: %s", cudaGetErrorString(err));
+        sphkv_set_error("%s: launch failed: %s", fn, cudaGetErrorString(err));
         return SPHKV_ERR_DEVICE;
     }
     return SPHKV_OK;
 }
+}  // namespace
 
 extern "C" sphkv_status sphkv_build_page_table(const uint8_t* tiers, int64_t n_entries, const int32_t* perm1,
                                                const int32_t* perm2, const int32_t* perm3, int32_t* table,

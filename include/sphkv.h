@@ -43,6 +43,8 @@
  *  T3 (3, 4, int4, 1984 B), or drop (no storage, excluded from the softmax).
  *  Page of tier t, in this order (all fields 16-byte aligned):
  *    r[16] fp16 | vscale[16] fp16 | code planes | value rows [16][16*v_bits]
+ *  The sign bit of r is the token's drop flag (see sphkv_set_keep); the
+ *  radius itself is the value with that bit cleared.
  *  Codes of a token are regrouped into 8 subtree blocks, block s for leaves
  *  8s..8s+7: L[s][j] = leaf code 8s+j; U[s][0..3] = level-1 nodes 4s..4s+3,
  *  U[s][4..5] = level-2 nodes 2s, 2s+1, U[s][6] = level-3 node s, U[s][7] =
@@ -166,6 +168,44 @@ sphkv_status sphkv_rdr_assign(const sphkv_cache* cache, const float* utility, co
                               void* stream);
 
 /*
+ * sphkv_rdr_rerun -- RDR again on a cache whose pages already hold codes, as
+ *   the context grows.  Spherical KV, AI Summary (retention allocates
+ *   precision and storage dynamically by estimated future utility).  Reading:
+ *   a page's codes can only be made coarser without the dense key, so each
+ *   unit chooses among its current tier and the coarser ones (drop included);
+ *   forced units (first n_sink, last n_recent pages) keep the finest tier they
+ *   are allowed (T1 if they are T1, else their current tier).  Otherwise
+ *   exactly sphkv_rdr_assign, with the same workspace.
+ *   tiers_io: [H_kv][total_pages] uint8, the current tiers on entry (every
+ *   page that holds tokens), the new ones on return.  Apply the result with
+ *   sphkv_build_page_table into new pools and sphkv_migrate.
+ */
+sphkv_status sphkv_rdr_rerun(const sphkv_cache* cache, const float* utility, const double* eps,
+                             int64_t budget_bytes, int32_t n_sink, int32_t n_recent, uint8_t* tiers_io,
+                             double* lambda_out, int64_t* bytes_out, void* workspace, size_t ws_bytes,
+                             int32_t* status_dev, void* stream);
+
+/*
+ * sphkv_migrate -- rewrite a cache's tokens into new pools after its tiers
+ *   changed (sphkv_rdr_rerun), transcoding from the stored codes alone; this
+ *   also compacts the pools to the new tier counts.  Reading (the pages give
+ *   no rule): each angle goes to the nearest point of the coarser grid,
+ *   computed exactly on the code integers with ties to even (leaf c ->
+ *   rne(c 2^b' / 2^b) mod 2^b', upper c -> rne(c (2^b' - 1) / (2^b - 1)));
+ *   the radius and its drop flag are kept; values are decoded (code x scale,
+ *   exact in fp64) and quantised again with the encoder's rule (new scale
+ *   fp16(max|v| / Q), codes clamp(rint(v / scale), -Q, Q)).  A token whose
+ *   tier does not change moves unchanged.  Bit-exact with a plain reference.
+ *   from: the old cache; to: the same sequences (B, H_kv, total_pages,
+ *   page_offsets, seq_lens) with the new page table and new pools, which the
+ *   caller zeroes first.  Every present token of every page `to` keeps is
+ *   written; pages `to` drops are skipped.  status_dev gets SPHKV_ERR_DATA
+ *   for a page that `to` makes finer than `from`, or keeps although `from`
+ *   dropped it (codes cannot be recovered), or a pool page out of range.
+ */
+sphkv_status sphkv_migrate(const sphkv_cache* from, const sphkv_cache* to, int32_t* status_dev, void* stream);
+
+/*
  * sphkv_build_page_table -- tiers -> page-table entries.
  *   Spherical KV, Abstract (each page holds one tier, with little metadata
  *   per page).  tiers: [n_entries] uint8 (0 drop, 1..3) in table order; the
@@ -215,8 +255,10 @@ sphkv_status sphkv_decode_attention(const sphkv_cache* cache, int32_t H_q, const
  *   - A cache whose scratch need (sphkv_decode_workspace_bytes with n_sm = 0)
  *     exceeds 4 MiB is rejected with SPHKV_ERR_ARG and a message naming both
  *     sizes; nothing is launched.
- *   - The first call on each device looks up the array's device address with
- *     that device current; make that first call before any stream capture.
+ *   - Every call looks up the array's device address with the caller's device
+ *     current (no allocation; the address stays right across a device reset).
+ *     The first call on a device also loads the library's kernels there: make
+ *     that first call before any stream capture.
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents (every value the kernels read is written earlier in the same
  *     call, so nothing needs clearing).  Calls whose work overlaps on the GPU,
@@ -250,6 +292,39 @@ size_t sphkv_decode_mq_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int
 sphkv_status sphkv_decode_attention_mq(const sphkv_cache* cache, int32_t n_q, int32_t H_q, const float* q,
                                        float* out, float* lse, void* workspace, size_t ws_bytes,
                                        int32_t* status_dev, void* stream);
+
+/*
+ * sphkv_set_keep -- per-token keep/drop inside kept pages.
+ *   Spherical KV, Abstract (RDR makes keep/drop decisions per token and
+ *   head).  Format: the sign bit of a token's stored radius is its drop flag
+ *   (a radius fp16(|k|) is never negative, so the bit is otherwise always 0):
+ *   decode skips a dropped token exactly as if it were absent (a head whose
+ *   tokens are all dropped gets out = 0, lse = -inf).  Page sizes do not
+ *   change; sphkv_encode writes tokens as kept.
+ *   keep: [H_kv][total_pages * 16] uint8, the layout of sphkv_rdr_assign's
+ *   utility (slot s of logical page i at i * 16 + s); nonzero = keep.  For
+ *   every present token (position < seq_len) of every page that is not
+ *   dropped, the flag is cleared (keep) or set (drop); other bytes are not
+ *   touched.  status_dev gets SPHKV_ERR_DATA for a pool page out of range.
+ */
+sphkv_status sphkv_set_keep(const sphkv_cache* cache, const uint8_t* keep, int32_t* status_dev, void* stream);
+
+/*
+ * sphkv_merge_partials -- combine decode results computed over disjoint parts
+ *   of the same sequences (split-KV across GPUs: each GPU decodes its own
+ *   contiguous range of a long stream's pages, then the parts are gathered).
+ *   Spherical KV, Abstract (long-context inference); the log-sum-exp combine
+ *   is the one sphkv_decode_attention uses for its own split pieces.  With
+ *   M = max_r lse_r and w_r = exp(lse_r - M):
+ *     out = sum_r w_r out_r / sum_r w_r,   lse = M + ln sum_r w_r.
+ *   A part with lse = -inf (no kept token) contributes nothing; a row whose
+ *   parts are all empty gets out = 0, lse = -inf.
+ *   out_parts: [n_parts][n_rows][128] fp32, lse_parts: [n_parts][n_rows] fp32
+ *   (e.g. n_rows = B * H_q for single-token decode), out: [n_rows][128],
+ *   lse: [n_rows].  1 <= n_parts <= 4096.  One kernel launch on `stream`.
+ */
+sphkv_status sphkv_merge_partials(const float* out_parts, const float* lse_parts, int32_t n_parts,
+                                  int64_t n_rows, float* out, float* lse, void* stream);
 
 #ifdef __cplusplus
 }

@@ -94,6 +94,36 @@ def oracle_unit(w: W.Workload, b: int, g: int, q, lens=None, tiers=None):
     return out[0], lse[0]
 
 
+def oracle_all_units(w: W.Workload, q, lens=None, tiers=None):
+    """Oracle attention of every (sequence, kv head) unit of w, over the
+    oracle's own encoding of the whole workload (the pool page ids do not
+    change the result).  Returns out [B, H_q, 128], lse [B, H_q]."""
+    ref = oracle_full_cache(w, lens=lens, tiers=tiers)
+    units = [(b, g) for b in range(w.B) for g in range(w.H_kv)]
+    ro, rl = oracle.cache_attention(ref, q, units)
+    return ro.reshape(w.B, w.H_q, -1), rl.reshape(w.B, w.H_q)
+
+
+def oracle_unit_dense(w: W.Workload, b: int, g: int, n: int, tiers):
+    """Keys and values of the first n tokens of sequence b, kv head g, as the
+    oracle encodes and decodes them (fp64), with the mask of kept tokens
+    (their page is not dropped).  Returns khat [n, 128], vhat [n, 128], keep."""
+    K, V = w.dense_rows(b, 0, n)
+    po = w.page_offsets
+    tok_tier = np.repeat(np.asarray(tiers)[g, po[b]:po[b] + (n + 15) // 16], 16)[:n]
+    khat = np.zeros((n, 128))
+    vhat = np.zeros((n, 128))
+    for t in (1, 2, 3):
+        idx = np.nonzero(tok_tier == t)[0]
+        if idx.size == 0:
+            continue
+        c = oracle.encode(K[idx, g], V[idx, g], t)
+        bl, bu, _ = oracle.TIER_BITS[t]
+        khat[idx] = oracle.decode_keys(c["leaf"], c["up"], c["r16"], bl, bu)
+        vhat[idx] = oracle.decode_values(c["vq"], c["s16"])
+    return khat, vhat, tok_tier != 0
+
+
 def assert_close(out_gpu, lse_gpu, out_ref, lse_ref, what=""):
     out_gpu = np.asarray(out_gpu, np.float64)
     lse_gpu = np.asarray(lse_gpu, np.float64)

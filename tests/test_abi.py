@@ -25,7 +25,7 @@ def test_library_exports_every_declared_symbol():
     build.build()
     lib = ctypes.CDLL(_lib.LIB_PATH)
     names = _declared()
-    assert len(names) == 11, names
+    assert len(names) == 15, names
     missing = [n for n in names if not hasattr(lib, n)]
     assert not missing, missing
     # the binding covers the same names

@@ -9,8 +9,8 @@ import pytest
 import oracle
 from compressed_paged_kv_ada_b200 import workloads as W
 
-from helpers import (assert_close, dense_torch, gpu_cache, oracle_full_cache, oracle_unit,
-                     to_torch)
+from helpers import (assert_close, dense_torch, gpu_cache, oracle_all_units, oracle_full_cache, oracle_unit,
+                     oracle_unit_dense, to_torch)
 
 pytestmark = pytest.mark.gpu
 
@@ -292,8 +292,9 @@ def _sampled_pages_bit_exact(w, cache, n_samples, rng):
 
 @pytest.mark.parametrize("name", ["llama32k", "ragged64", "long512k"])
 def test_full_size_workloads(name):
-    """Full-size workloads: sampled pages bit-exact, sampled units' decode
-    within tolerance of the oracle, page table equal to the oracle's."""
+    """Full-size workloads: sampled pages bit-exact, the page table equal to
+    the oracle's, and the decode of every (sequence, kv head) unit within
+    tolerance of the oracle."""
     w = W.make(name)
     cache = gpu_cache(w)
     assert np.array_equal(cache.page_table.cpu().numpy(), oracle.build_page_table(w.tiers, w.pool_perms()))
@@ -301,13 +302,13 @@ def test_full_size_workloads(name):
     _sampled_pages_bit_exact(w, cache, 40, rng)
     q = w.queries()
     out, lse = _decode(cache, q)
+    del cache
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
-    units = {(0, 0), (w.B - 1, w.H_kv - 1)}
-    while len(units) < (4 if name == "long512k" else 6):
-        units.add((int(rng.integers(w.B)), int(rng.integers(w.H_kv))))
-    for b, g in sorted(units):
-        ro, rl = oracle_unit(w, b, g, q)
-        assert_close(out[b, 4 * g:4 * g + 4], lse[b, 4 * g:4 * g + 4], ro, rl, f"{name} unit {(b, g)}")
+    ro, rl = oracle_all_units(w, q)
+    for b in range(w.B):
+        for g in range(w.H_kv):
+            rows = slice(4 * g, 4 * g + 4)
+            assert_close(out[b, rows], lse[b, rows], ro[b, rows], rl[b, rows], f"{name} unit {(b, g)}")
 
 
 # ------------------------------------------------------------------- RDR --
@@ -344,8 +345,11 @@ def test_rdr_infeasible_budget_reports():
 
 def test_e2e_rdr_full():
     """End-to-end: 16 x 32768 prefill, RDR at 25 % of the fp16 bytes (tiers
-    bit-exact vs the oracle), encode into the chosen tiers, then appends with
-    decode; sampled steps and units against the oracle."""
+    bit-exact vs the oracle), encode into the chosen tiers, then 256 steps of
+    append + decode.  Against the oracle: every unit at steps 0, 1 and 255,
+    and every step for sequences 0 and 1."""
+    from concurrent.futures import ThreadPoolExecutor
+
     torch = _torch()
     w = W.make("e2e_rdr")
     util = w.utility()
@@ -367,25 +371,56 @@ def test_e2e_rdr_full():
                      torch.arange(n, dtype=torch.int32, device="cuda"))
     cache.check()
     steps = w.extra["steps"]
-    lens = w.seq_lens.copy()
-    rng = np.random.default_rng(5)
-    check_steps = {0, 1, steps - 1}
+    prefill = w.seq_lens.copy()
+    lens = prefill.copy()
+    full_steps = (0, 1, steps - 1)
+    got_full, got_seq01 = {}, []
+    # the appended rows of every sequence, drawn once (a row is the same
+    # whichever slice it is drawn in)
+    app = [w.dense_rows(b, int(prefill[b]), int(prefill[b]) + steps) for b in range(w.B)]
     for step in range(steps):
-        rows = [w.dense_rows(b, int(lens[b]), int(lens[b]) + 1) for b in range(w.B)]
-        Kd, Vd = dense_torch(w, np.concatenate([r[0] for r in rows]), np.concatenate([r[1] for r in rows]))
+        Kd, Vd = dense_torch(w, np.stack([a[0][step] for a in app]), np.stack([a[1][step] for a in app]))
         cache.encode(Kd, Vd, torch.arange(w.B, dtype=torch.int32, device="cuda"),
                      to_torch(lens.astype(np.int32)))
         lens += 1
         cache.seq_lens.copy_(to_torch(lens.astype(np.int32)))
-        q = w.queries(step + 1)
-        out, lse = cache.decode(to_torch(q, torch.float32))
-        if step in check_steps:
+        out, lse = cache.decode(to_torch(w.queries(step + 1), torch.float32))
+        if step in full_steps:
             cache.check()
-            out, lse = out.cpu().numpy(), lse.cpu().numpy()
-            for b, g in [(0, 0), (1, 3), (int(rng.integers(w.B)), int(rng.integers(w.H_kv)))]:
-                ro, rl = oracle_unit(w, b, g, q, lens=lens, tiers=tiers)
-                assert_close(out[b, 4 * g:4 * g + 4], lse[b, 4 * g:4 * g + 4], ro, rl, f"step {step} {(b, g)}")
+            got_full[step] = (out.cpu().numpy(), lse.cpu().numpy())
+        got_seq01.append((out[:2].cpu().numpy(), lse[:2].cpu().numpy()))
     cache.check()
+    del cache
+    # every unit at steps 0, 1, 255
+    for step in full_steps:
+        o, l = got_full[step]
+        ro, rl = oracle_all_units(w, w.queries(step + 1), lens=prefill + step + 1, tiers=tiers)
+        for b in range(w.B):
+            for g in range(w.H_kv):
+                rs = slice(4 * g, 4 * g + 4)
+                assert_close(o[b, rs], l[b, rs], ro[b, rs], rl[b, rs], f"step {step} unit {(b, g)}")
+    # every step for sequences 0 and 1: each unit's keys decoded once and its
+    # kept tokens packed in position order, so the prefix a step saw is a
+    # contiguous slice (no copy); then dense attention over that prefix
+    dense = {}
+    for b in (0, 1):
+        for g in range(w.H_kv):
+            kh, vh, keep = oracle_unit_dense(w, b, g, int(lens[b]), tiers)
+            dense[(b, g)] = (np.ascontiguousarray(kh[keep]), np.ascontiguousarray(vh[keep]), np.cumsum(keep))
+    qs = [np.asarray(w.queries(step + 1), np.float64) for step in range(steps)]
+
+    def ref(item):
+        step, b, g = item
+        kk, vk, n_kept = dense[(b, g)]
+        m = int(n_kept[int(prefill[b]) + step])   # kept tokens among the first prefill + step + 1
+        return item, oracle.attention(kk[:m], vk[:m], qs[step][b, 4 * g:4 * g + 4])
+
+    items = [(step, b, g) for step in range(steps) for b in (0, 1) for g in range(w.H_kv)]
+    with ThreadPoolExecutor(max_workers=max(1, oracle.num_threads())) as ex:
+        for (step, b, g), (ro, rl) in ex.map(ref, items):
+            o, l = got_seq01[step]
+            rs = slice(4 * g, 4 * g + 4)
+            assert_close(o[b, rs], l[b, rs], ro, rl, f"step {step} unit {(b, g)}")
 
 
 # ---------------------------------------------------------------- errors --

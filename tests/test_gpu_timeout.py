@@ -3,8 +3,9 @@ context stays usable afterwards.
 
 The test loads libsphkv_testhooks.so: the same library with decode.cu built
 with SPHKV_TEST_HOOKS.  With SPHKV_TEST_SKIP_FIRST_COPY set, warp 0 of CTA 0
-skips its first page copy, so its (shortened) wait for that page runs out;
-nothing faults and no wait is unbounded.  The product library is built without
+skips its first page copy and waits for it with a shortened limit, so that
+wait runs out; every other warp and CTA runs as in the product library.
+Nothing faults and no wait is unbounded.  The product library is built without
 the flag.
 """
 import ctypes
@@ -41,14 +42,20 @@ def test_page_wait_timeout_reports_and_context_recovers(monkeypatch):
         assert code == _lib.OK, T.sphkv_last_error()
         torch.cuda.synchronize()
 
+    ref_out, ref_lse = cache.decode(q)
+    cache.check()
     monkeypatch.setenv("SPHKV_TEST_SKIP_FIRST_COPY", "1")
     run()
     assert int(status.item()) == _lib.ERR_TIMEOUT
+    # Only CTA 0 stopped.  Its pages all lie in unit (0, 0): that unit holds the
+    # first 129 of the 446 pages, and with at least 4 CTAs (min(7, SM count))
+    # CTA 0 takes at most 112 of them.  Every other unit is exact.
+    for b, g in [(0, 1), (1, 0), (1, 1)]:
+        rows = slice(4 * g, 4 * g + 4)
+        assert torch.equal(out[b, rows], ref_out[b, rows]) and torch.equal(lse[b, rows], ref_lse[b, rows])
     # the context is still usable: the next call (no skipped copy) is correct
     monkeypatch.delenv("SPHKV_TEST_SKIP_FIRST_COPY")
     status.zero_()
     run()
     assert int(status.item()) == _lib.OK
-    ref_out, ref_lse = cache.decode(q)
-    cache.check()
     assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
