@@ -57,25 +57,26 @@ constexpr int kPartStride = 132;    // floats per (slot, head): m, l, pad, pad, 
 
 // Cos/sin tables, shared by both decode kernels.  T1: one 256-byte row per
 // code, [leaf (cos,sin) x 16 lane replicas][upper (cos,sin) x 16 replicas].
-// T2, T3: upper grid only, one 128-byte row of 16 replicas per code.  T2 and
-// T3 leaves read T1 leaf rows or the query-folded table: the leaf grids nest
-// (T2 code c has the angle of T1 code 16c, T3 code c that of T2 code 2c).
+// T2, T3: upper grid only, 16 replicas (128 bytes) per code, in 128-byte (T2)
+// or 256-byte (T3) rows.  T2 and T3 leaves read the query-folded tables, built
+// from T1 leaf rows: the leaf grids nest (T2 code c has the angle of T1 code
+// 16c, T3 code c that of T2 code 2c).
 //
-// Shared-memory layout of decode_kernel<NQ>.  Region offsets are taken from a
-// zero point: for one query token (NQ = 1) that is shared address 0, i.e. the
-// offsets are absolute shared-window addresses, each table aligned to its own
-// size so that a lookup address is the OR of the table base, the code and the
-// lane's replica (one instruction per code, no address add); the dynamic block
-// must then start below the first region, which the kernel checks.  For a pair
-// of query tokens (NQ = 2) the zero point is the start of the dynamic block.
+// Shared-memory layout of decode_kernel<NQ>.  Region offsets are absolute
+// shared-window addresses (the dynamic block must start below the first
+// region, which the kernel checks), each table placed so that a lookup address
+// is the code permuted or OR-ed into the table base and the lane's replica,
+// plus an immediate offset: one or two instructions per code, no address add.
 template <int NQ>
 struct Layout;
 // One query token: 12 warps, 8 lanes per token, each lane holding its
 // subtree's query slice in registers (168 registers a thread); two-stage page
 // rings.  The query-folded T2/T3 leaf table holds, for leaf j = 8s + i and T2
 // code c, the 4 heads' q[2j] cos(phi_c) + q[2j+1] sin(phi_c) (times the logit
-// scale) at kFold + (c << 11) + 144 s + 16 i, in the head order of the lanes
-// that own subtree s.
+// scale) at kFold + (i << 12) + (c << 8) + (s << 4), in the head order of the
+// lanes that own subtree s: a code byte placed in bits 8..15 of the lane's
+// base (s << 4) is the address, leaf i's slab an immediate offset, and the 8
+// lanes of a token read 8 distinct bank groups.
 template <>
 struct Layout<1> {
     static constexpr int kWarps = 12;
@@ -83,35 +84,42 @@ struct Layout<1> {
     static constexpr int kHeads = kG;
     static constexpr int kPbufFloats = 16 * kG + 2 * kG;   // p*scale per (token, head); alpha per head; valid
     static constexpr uint32_t kUpT2 = 8192;                // 64 rows x 128 B, 8 KB aligned
-    static constexpr uint32_t kUpT3 = 16384;               // 16 rows x 128 B, 2 KB aligned
-    static constexpr uint32_t kPbuf = 18432;
+    static constexpr uint32_t kUpT3 = 16384;               // 16 rows x 256 B (128 B used)
+    static constexpr uint32_t kPbuf = 20480;
     static constexpr uint32_t kBar = kPbuf + kWarps * kPbufFloats * 4;
     static constexpr uint32_t kSlice = kBar + kWarps * kStages * 8;
-    static constexpr uint32_t kFold = 32768;               // 16 codes x 2 KB, 32 KB aligned
+    static constexpr uint32_t kFold = 32768;               // 8 leaf slabs x 16 codes x 256 B
     static constexpr uint32_t kT1 = 65536;                 // 256 rows x 256 B, 64 KB aligned
     static constexpr uint32_t kStage = 131072;
     static constexpr int kSmemBytes = (int)(kStage + kWarps * kStages * kStageBytes);
 };
-// A pair of query tokens (8 heads): 16 warps, two-stage rings; the pair's
-// query rows (4 arrays of (q[2j], q[2j+1]) for heads 2a, 2a+1, at byte
-// 1024 a + (144 s ^ 16 i) for leaf j = 8s + i) sit in shared memory.
+// A pair of query tokens (8 heads): the same absolute plan and lane mapping as
+// one query, 12 warps, no query registers.  Lane (k, s) holds, for its subtree
+// s, slots i = 0..7 of the unit's 8 heads in the order head(i) = i ^ s (heads
+// 0-3: the first query token, 4-7: the second), so that the 8-lane sum leaves
+// lane s with head s.  T1 leaves read the query rows kQ (slot pair hp = slots
+// 2hp, 2hp+1 of leaf j = 8s + i at kQ + 512 i + 128 hp + 16 s); T2/T3 leaves
+// read slots 0-3 from the first folded table and 4-7 from the second (entry of
+// T2 code c: kFold + (i << 12) + (c << 8) + (s << 4), the second table's 128
+// bytes on).
 template <>
 struct Layout<2> {
-    static constexpr int kWarps = 16;
+    static constexpr int kWarps = 12;
     static constexpr int kStages = 2;
     static constexpr int kHeads = 2 * kG;
-    static constexpr int kPbufFloats = 16 * 2 * kG + 2 * 2 * kG;   // weights; alpha; valid counts
-    static constexpr uint32_t kT1 = 0;
-    static constexpr uint32_t kUpT2 = 256 * 256;
-    static constexpr uint32_t kUpT3 = kUpT2 + 64 * 128;
-    static constexpr uint32_t kStage = kUpT3 + 16 * 128;
-    static constexpr uint32_t kQ = kStage + kWarps * kStages * kStageBytes;
-    static constexpr uint32_t kPbuf = kQ + 4 * 1024;
+    static constexpr int kPbufFloats = 16 * 2 * kG + 2 * 2 * kG;   // weights; alpha per head
+    static constexpr uint32_t kUpT2 = 8192;
+    static constexpr uint32_t kUpT3 = 16384;
+    static constexpr uint32_t kPbuf = 20480;
     static constexpr uint32_t kBar = kPbuf + kWarps * kPbufFloats * 4;
     static constexpr uint32_t kSlice = kBar + kWarps * kStages * 8;
-    static constexpr int kSmemBytes = (int)(kSlice + kWarps * 4);
+    static constexpr uint32_t kQ = 27648;                  // 8 leaves x 4 slot pairs x 8 subtrees x 16 B
+    static constexpr uint32_t kFold = 32768;               // 8 leaf slabs x 16 codes x 2 tables x 128 B
+    static constexpr uint32_t kFold2 = 128;                // second table, from the first
+    static constexpr uint32_t kT1 = 65536;
+    static constexpr uint32_t kStage = 131072;
+    static constexpr int kSmemBytes = (int)(kStage + kWarps * kStages * kStageBytes);
 };
-constexpr int kLutT1 = 0, kLutT2 = Layout<2>::kUpT2, kLutT3 = Layout<2>::kUpT3;   // pair kernel, relative
 template <int NQ>
 constexpr bool layout_ok()
 {
@@ -126,7 +134,11 @@ static_assert(layout_ok<1>() && layout_ok<2>(), "shared-memory layout");
 static_assert(Layout<1>::kSlice + Layout<1>::kWarps * 4 <= Layout<1>::kFold && Layout<1>::kFold % 32768 == 0 &&
                   Layout<1>::kFold + 32768 <= Layout<1>::kT1 && Layout<1>::kT1 + 65536 <= Layout<1>::kStage,
               "one-query regions");
-static_assert(Layout<2>::kQ % 128 == 0, "pair query rows");
+static_assert(Layout<2>::kSlice + Layout<2>::kWarps * 4 <= Layout<2>::kQ && Layout<2>::kQ % 128 == 0 &&
+                  Layout<2>::kQ + 4096 <= Layout<2>::kFold && Layout<2>::kFold % 32768 == 0 &&
+                  Layout<2>::kFold + 32768 <= Layout<2>::kT1 &&
+                  Layout<2>::kT1 + 65536 <= Layout<2>::kStage && Layout<1>::kUpT2 == Layout<2>::kUpT2,
+              "pair regions");
 
 constexpr float kLn2 = 0.6931471805599453f;
 // log2(e) / sqrt(128): logits are kept in the log2 domain
@@ -327,54 +339,10 @@ __device__ __forceinline__ float pow2_floor(float x)
     return __int_as_float(__float_as_int(x) & 0x7f800000);
 }
 
-// Table offsets of the 8 leaf and 8 upper codes of one subtree block.  Leaves
-// (every tier) index T1 leaf rows: T1 code c at c << 8, T2 code c at c << 12
-// (T1 row 16c), T3 code c at c << 13 (T1 row 32c).  Upper codes: T1 c << 8
-// (the upper half is 128 bytes into the row), T2/T3 c << 7 into their own
-// 128-byte rows.  rep = (lane & 15) << 3 picks the lane's replica, so a half
-// warp's 64-bit lookups never share a bank.
 template <int T>
 __device__ __forceinline__ uint32_t shift_mask(uint32_t x, int sh, uint32_t mask)
 {
     return (sh >= 0 ? x << sh : x >> -sh) & mask;
-}
-
-template <int T>
-__device__ __forceinline__ void block_offsets(const uint8_t* codes, int blk, uint32_t rep, uint32_t (&lo)[8],
-                                              uint32_t (&uo)[8])
-{
-    if (T == 1) {   // byte codes: one permute places the code in bits 8..15
-        const uint4 w = *(const uint4*)(codes + blk * 16);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            lo[j] = __byte_perm(w.x, rep, 0x7604 | (j << 4));
-            lo[4 + j] = __byte_perm(w.y, rep, 0x7604 | (j << 4));
-            uo[j] = __byte_perm(w.z, rep, 0x7604 | (j << 4));
-            uo[4 + j] = __byte_perm(w.w, rep, 0x7604 | (j << 4));
-        }
-    } else if (T == 2) {   // leaf nibbles; upper code j = bits 6j..6j+5 of the 48-bit field h:w.y
-        const uint2 w = *(const uint2*)(codes + blk * 8);
-        const uint32_t h = *(const uint16_t*)(codes + kP * 64 + blk * 2);
-        constexpr uint32_t kUpMask = 63u << 7;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) lo[j] = shift_mask<T>(w.x, 12 - 4 * j, 15u << 12) | rep;
-        uo[0] = ((w.y << 7) & kUpMask) | rep;
-        uo[1] = ((w.y << 1) & kUpMask) | rep;
-        uo[2] = ((w.y >> 5) & kUpMask) | rep;
-        uo[3] = ((w.y >> 11) & kUpMask) | rep;
-        uo[4] = ((w.y >> 17) & kUpMask) | rep;
-        uo[5] = (__funnelshift_r(w.y, h, 23) & kUpMask) | rep;
-        uo[6] = ((h << 3) & kUpMask) | rep;
-        uo[7] = ((h >> 3) & kUpMask) | rep;
-    } else {   // upper nibbles; leaf code j = bits 3j..3j+2 of the 24-bit field l8:l16
-        const uint32_t u = *(const uint32_t*)(codes + blk * 4);
-        const uint32_t lf = *(const uint16_t*)(codes + kP * 32 + blk * 2) | ((uint32_t)codes[kP * 48 + blk] << 16);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            lo[j] = shift_mask<T>(lf, 13 - 3 * j, 7u << 13) | rep;
-            uo[j] = shift_mask<T>(u, 7 - 4 * j, 15u << 7) | rep;
-        }
-    }
 }
 
 // 2^x on the special-function unit (max relative error about 2^-22); -inf -> 0.
@@ -401,21 +369,13 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Table offset of upper code 7 (the block's top node) of one subtree block.
-template <int T>
-__device__ __forceinline__ uint32_t block_top(const uint8_t* codes, int blk, uint32_t base_rep)
-{
-    if (T == 1) return __byte_perm(*(const uint32_t*)(codes + blk * 16 + 12), base_rep, 0x7634);
-    if (T == 2) return ((*(const uint16_t*)(codes + kP * 64 + blk * 2) >> 3) & (63u << 7)) | base_rep;
-    return (((*(const uint32_t*)(codes + blk * 4)) >> 28) << 7) | base_rep;
-}
-
 // Shared-memory loads by 32-bit shared address (the lookups below build full
 // addresses; these keep the compiler from adding a base to each).
+template <int Off = 0>
 __device__ __forceinline__ float lds32(uint32_t a)
 {
     float v;
-    asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+    asm("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(a), "n"(Off));
     return v;
 }
 template <int Off = 0>
@@ -433,12 +393,15 @@ __device__ __forceinline__ float4 lds128(uint32_t a)
     return v;
 }
 
-// Full shared addresses of the 8 leaf and 8 upper lookups of one subtree
-// block, for the one-query layout.  rep1 = kT1 | leaf replica, repU = the
-// tier's upper table (kT1 for T1) | upper replica, fb = kFold | 144 s.  T1:
-// row addresses (the upper half of a row is 128 bytes on).  T2/T3 leaves: the query-folded entry of
-// leaf 0 of the block for that code (leaf i is 16 i bytes on; T3 code c is
-// T2 code 2c).
+// Shared addresses (before the immediate offset of the table) of the 8 leaf
+// and 8 upper lookups of one subtree block.  rep1 = kT1 | leaf replica; repU
+// = the upper table (kT1 for T1, kUpT2 for T2, none for T3) | upper replica;
+// fb = the lane's folded-table column (s << 4).  T1: row addresses, the code
+// byte permuted into bits 8..15 (the upper half of a row is 128 bytes on).
+// T2 leaves and T3 uppers: 4-bit codes, masked into bytes and permuted into
+// bits 8..15 the same way (T3 upper rows are 256 bytes apart).  T3 leaves:
+// code c is T2 code 2c, shifted to bit 9.  T2 uppers: 6-bit codes of a 48-bit
+// field, one 128-byte row each.
 template <int T>
 __device__ __forceinline__ void block_addrs(const uint8_t* codes, int blk, uint32_t rep1, uint32_t repU,
                                             uint32_t fb, uint32_t (&lo)[8], uint32_t (&uo)[8])
@@ -455,9 +418,13 @@ __device__ __forceinline__ void block_addrs(const uint8_t* codes, int blk, uint3
     } else if (T == 2) {   // leaf nibbles; upper code j = bits 6j..6j+5 of the 48-bit field h:w.y
         const uint2 w = *(const uint2*)(codes + blk * 8);
         const uint32_t h = *(const uint16_t*)(codes + kP * 64 + blk * 2);
-        constexpr uint32_t kUpMask = 63u << 7;
+        const uint32_t even = w.x & 0x0F0F0F0Fu, odd = (w.x >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) lo[j] = shift_mask<T>(w.x, 11 - 4 * j, 15u << 11) | fb;
+        for (int k = 0; k < 4; ++k) {
+            lo[2 * k] = __byte_perm(even, fb, 0x7604 | (k << 4));
+            lo[2 * k + 1] = __byte_perm(odd, fb, 0x7604 | (k << 4));
+        }
+        constexpr uint32_t kUpMask = 63u << 7;
         uo[0] = ((w.y << 7) & kUpMask) | repU;
         uo[1] = ((w.y << 1) & kUpMask) | repU;
         uo[2] = ((w.y >> 5) & kUpMask) | repU;
@@ -469,11 +436,14 @@ __device__ __forceinline__ void block_addrs(const uint8_t* codes, int blk, uint3
     } else {   // upper nibbles; leaf code j = bits 3j..3j+2 of the 24-bit field l8:l16
         const uint32_t u = *(const uint32_t*)(codes + blk * 4);
         const uint32_t lf = *(const uint16_t*)(codes + kP * 32 + blk * 2) | ((uint32_t)codes[kP * 48 + blk] << 16);
+        const uint32_t even = u & 0x0F0F0F0Fu, odd = (u >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            lo[j] = shift_mask<T>(lf, 12 - 3 * j, 7u << 12) | fb;
-            uo[j] = shift_mask<T>(u, 7 - 4 * j, 15u << 7) | repU;
+        for (int k = 0; k < 4; ++k) {
+            uo[2 * k] = __byte_perm(even, repU, 0x7604 | (k << 4));
+            uo[2 * k + 1] = __byte_perm(odd, repU, 0x7604 | (k << 4));
         }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) lo[j] = shift_mask<T>(lf, 9 - 3 * j, 7u << 9) | fb;
     }
 }
 
@@ -504,12 +474,13 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, int lane, const f
     const int s = lane & 7;
     const uint32_t rep = (uint32_t)(lane & 15) << 3;
     const uint32_t rep1 = L::kT1 | rep;
-    const uint32_t repU = (T == 1 ? L::kT1 : T == 2 ? L::kUpT2 : L::kUpT3) | rep;
-    const uint32_t fb = L::kFold | (144u * (uint32_t)s);
-    constexpr int kUp = T == 1 ? 128 : 0;   // upper (cos, sin) inside a T1 row
+    const uint32_t repU = (T == 1 ? L::kT1 : T == 2 ? L::kUpT2 : 0u) | rep;
+    const uint32_t fb = (uint32_t)s << 4;
+    // immediate offset of the upper (cos, sin): inside a T1 row, or the T3 table
+    constexpr int kUp = T == 1 ? 128 : T == 2 ? 0 : (int)L::kUpT3;
     // own side at levels 4, 5 and the root (the upper half of a T1 row)
-    const uint32_t side4 = kUp + ((uint32_t)(s & 1) << 2), side5 = kUp + ((uint32_t)((s >> 1) & 1) << 2),
-                   side6 = kUp + ((uint32_t)(s >> 2) << 2);
+    const uint32_t side4 = (uint32_t)(s & 1) << 2, side5 = (uint32_t)((s >> 1) & 1) << 2,
+                   side6 = (uint32_t)(s >> 2) << 2;
     const int grp = lane & ~7;
     const uint8_t* codes = pg + Tier<1>::f.off_codes;
 #pragma unroll
@@ -522,11 +493,12 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, int lane, const f
         const uint32_t o5 = __shfl_sync(full, uo[7], grp + 4 + (s >> 2));
         const uint32_t o6 = __shfl_sync(full, uo[7], grp + 6);
         // radius bits: the sign bit is the token's drop flag, the rest the radius
+        // (a flagged token's logit is replaced by -inf, so its sign is left in)
         const uint32_t rb = ((const uint16_t*)pg)[t];
-        float v = __half2float(__ushort_as_half((unsigned short)(rb & 0x7fffu)));
-        v *= lds32(o6 | side6);
-        v *= lds32(o5 | side5);
-        v *= lds32(o4 | side4);
+        float v = __half2float(__ushort_as_half((unsigned short)rb));
+        v *= lds32<kUp>(o6 | side6);
+        v *= lds32<kUp>(o5 | side5);
+        v *= lds32<kUp>(o4 | side4);
         float w2[2], w1[4], wl[8];
         {
             const float2 f = lds64<kUp>(uo[6]);
@@ -563,15 +535,15 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, int lane, const f
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 float4 F;
-                switch (j) {   // leaf j of the block is 16 j bytes on
-                case 0: F = lds128<0>(lo[j]); break;
-                case 1: F = lds128<16>(lo[j]); break;
-                case 2: F = lds128<32>(lo[j]); break;
-                case 3: F = lds128<48>(lo[j]); break;
-                case 4: F = lds128<64>(lo[j]); break;
-                case 5: F = lds128<80>(lo[j]); break;
-                case 6: F = lds128<96>(lo[j]); break;
-                default: F = lds128<112>(lo[j]); break;
+                switch (j) {   // leaf j's slab is 4 KB on
+                case 0: F = lds128<L::kFold>(lo[j]); break;
+                case 1: F = lds128<L::kFold + 4096>(lo[j]); break;
+                case 2: F = lds128<L::kFold + 8192>(lo[j]); break;
+                case 3: F = lds128<L::kFold + 12288>(lo[j]); break;
+                case 4: F = lds128<L::kFold + 16384>(lo[j]); break;
+                case 5: F = lds128<L::kFold + 20480>(lo[j]); break;
+                case 6: F = lds128<L::kFold + 24576>(lo[j]); break;
+                default: F = lds128<L::kFold + 28672>(lo[j]); break;
                 }
                 const float2 ww = make_float2(wl[j], wl[j]);
                 acc01 = j == 0 ? __fmul2_rn(ww, make_float2(F.x, F.y)) : __ffma2_rn(ww, make_float2(F.x, F.y), acc01);
@@ -777,111 +749,134 @@ __device__ __forceinline__ void process_page(const uint8_t* pg, int tier, int va
 // ---------------------------------------------- two query tokens per pass --
 // Several decode query tokens per sequence (speculative or chunked decode):
 // a launch takes a pair of them, i.e. 8 query heads per kv head, so one page
-// stream serves both and the tensor-core tile's 8 columns are all used.  The
-// pair's query rows sit in shared memory (Layout<2>: 4 arrays of (q[2j],
-// q[2j+1]) for heads 2a, 2a+1, at byte 1024 a + (144 s ^ 16 i) for leaf
-// j = 8s + i); every tier's leaves read (cos, sin) from the T1 leaf rows.
+// stream, one code unpack and one set of path products serve both tokens,
+// and the tensor-core tile's 8 columns are all used.
 constexpr int kGQ2 = 2 * kG;                          // heads per unit
 
-// One subtree block for the 8 heads of a query pair, top down from its
-// weight v: per head, (q[2j], q[2j+1]) . (w cos phi, w sin phi) summed in
-// f32x2 (even, odd) pairs.
+// Logits of the 16 tokens of one page for the 8 heads of a query pair, in
+// the log2 domain: lane (k4, s) ends with lg[pass] = the logit of token
+// 4 pass + k4 for head s.  The lane mapping, the code unpack and the path
+// products are page_logits'; the leaf terms go to 8 slots (slot i: head i ^ s).
+// T1: (w cos phi, w sin phi) times the 8 slots' query pairs, four 16-byte
+// rows in shared memory (the four token groups of the warp read the same
+// rows).  T2/T3: one 16-byte lookup in each of the two folded tables.  The 8-lane sum is a select-free reduce-scatter
+// (xor 4, 2, 1): after it lane s holds head s.
 template <int T>
-__device__ __forceinline__ void subtree_mq(float v, const uint32_t (&lo)[8], const uint32_t (&uo)[8],
-                                           const uint8_t* smem, const uint8_t* lut_up, const uint32_t (&fl)[8],
-                                           float2 (&acc2)[kGQ2], bool first)
+__device__ __forceinline__ void page_logits_pair(const uint8_t* pg, int lane, float (&lg)[4])
 {
-    float w2[2], w1[4], wl[8];
-    {
-        const float2 f = *(const float2*)(lut_up + uo[6]);
-        w2[0] = v * f.x;
-        w2[1] = v * f.y;
-    }
-#pragma unroll
-    for (int n = 0; n < 2; ++n) {
-        const float2 f = *(const float2*)(lut_up + uo[4 + n]);
-        w1[2 * n] = w2[n] * f.x;
-        w1[2 * n + 1] = w2[n] * f.y;
-    }
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const float2 f = *(const float2*)(lut_up + uo[m]);
-        wl[2 * m] = w1[m] * f.x;
-        wl[2 * m + 1] = w1[m] * f.y;
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const float2 f = *(const float2*)(smem + kLutT1 + lo[j]);
-        const float2 kk = make_float2(wl[j] * f.x, wl[j] * f.y);
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            const float4 qv = *(const float4*)(smem + Layout<2>::kQ + 1024 * a + fl[j]);   // heads 2a, 2a+1
-            const float2 qa = make_float2(qv.x, qv.y), qb = make_float2(qv.z, qv.w);
-            acc2[2 * a] = (first && j == 0) ? __fmul2_rn(qa, kk) : __ffma2_rn(qa, kk, acc2[2 * a]);
-            acc2[2 * a + 1] = (first && j == 0) ? __fmul2_rn(qb, kk) : __ffma2_rn(qb, kk, acc2[2 * a + 1]);
-        }
-    }
-}
-
-// Logits of the 16 tokens of one page for the 8 heads of a query pair, into
-// pbuf[t * 8 + head]; the lane mapping is page_logits' (4 lanes per token,
-// blocks 2q, 2q+1), and the butterfly leaves lane q with heads 2q, 2q+1.
-template <int T>
-__device__ __forceinline__ void page_logits_mq(const uint8_t* pg, const uint8_t* smem, float* pbuf, int lane,
-                                               const uint32_t (&flA)[8])
-{
+    using L = Layout<2>;
     const unsigned full = 0xffffffffu;
-    const int q = lane & 3, k8 = lane >> 2;
-    const bool a_right = k8 & 1;
-    const int sA = 2 * q + (k8 & 1), sB = sA ^ 1;
-    constexpr int kBase = T == 1 ? kLutT1 : T == 2 ? kLutT2 : kLutT3;
-    constexpr int kUp = T == 1 ? 128 : 0;
-    const uint8_t* lut_up = smem + kBase + kUp;
+    const int s = lane & 7;
     const uint32_t rep = (uint32_t)(lane & 15) << 3;
+    const uint32_t rep1 = L::kT1 | rep;
+    const uint32_t repU = (T == 1 ? L::kT1 : T == 2 ? L::kUpT2 : 0u) | rep;
+    const uint32_t fb = (uint32_t)s << 4;
+    const uint32_t qb = L::kQ | ((uint32_t)s << 4);
+    constexpr int kUp = T == 1 ? 128 : T == 2 ? 0 : (int)L::kUpT3;
+    const uint32_t side4 = (uint32_t)(s & 1) << 2, side5 = (uint32_t)((s >> 1) & 1) << 2,
+                   side6 = (uint32_t)(s >> 2) << 2;
+    const int grp = lane & ~7;
     const uint8_t* codes = pg + Tier<1>::f.off_codes;
-    uint32_t flB[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) flB[i] = flA[i] ^ 144u;
-    const uint32_t side6 = (uint32_t)(q >> 1) << 2, side5 = (uint32_t)(q & 1) << 2;
-    const int base = lane & ~3;
-#pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-        const int t = pass * 8 + k8;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int t = pass * 4 + (lane >> 3);
         uint32_t lo[8], uo[8];
-        block_offsets<T>(codes, t * 8 + sA, rep, lo, uo);
-        const uint32_t topB = block_top<T>(codes, t * 8 + sB, rep);
-        const uint32_t top2 = (a_right ? topB : uo[7]) | ((a_right ? uo[7] : topB) << 16);
-        const uint32_t w4 = __shfl_sync(full, top2, base + (q >> 1));
-        const uint32_t w5 = __shfl_sync(full, top2, base + 2);
-        const uint32_t w6 = __shfl_sync(full, top2, base + 3);
-        const uint32_t o4 = (w4 >> (16 * (q & 1))) & 0xffffu;
-        const uint32_t o5 = (w5 >> (16 * (q >> 1))) & 0xffffu;
-        const uint32_t o6 = w6 & 0xffffu;
+        block_addrs<T>(codes, pass * 32 + lane, rep1, repU, fb, lo, uo);
+        const uint32_t o4 = __shfl_sync(full, uo[7], grp + (s >> 1));
+        const uint32_t o5 = __shfl_sync(full, uo[7], grp + 4 + (s >> 2));
+        const uint32_t o6 = __shfl_sync(full, uo[7], grp + 6);
         const uint32_t rb = ((const uint16_t*)pg)[t];   // the sign bit is the token's drop flag
-        float v = __half2float(__ushort_as_half((unsigned short)(rb & 0x7fffu))) * kLogitScale;
-        v *= *(const float*)(lut_up + o6 + side6);
-        v *= *(const float*)(lut_up + o5 + side5);
-        const float2 f4 = *(const float2*)(lut_up + o4);
-        const float vA = v * (a_right ? f4.y : f4.x), vB = v * (a_right ? f4.x : f4.y);
-        float2 acc2[kGQ2];
-        subtree_mq<T>(vA, lo, uo, smem, lut_up, flA, acc2, true);
-        block_offsets<T>(codes, t * 8 + sB, rep, lo, uo);
-        subtree_mq<T>(vB, lo, uo, smem, lut_up, flB, acc2, false);
-        float acc[kGQ2];
+        float v = __half2float(__ushort_as_half((unsigned short)rb));
+        v *= lds32<kUp>(o6 | side6);
+        v *= lds32<kUp>(o5 | side5);
+        v *= lds32<kUp>(o4 | side4);
+        float w2[2], w1[4], wl[8];
+        {
+            const float2 f = lds64<kUp>(uo[6]);
+            w2[0] = v * f.x;
+            w2[1] = v * f.y;
+        }
 #pragma unroll
-        for (int h = 0; h < kGQ2; ++h) acc[h] = acc2[h].x + acc2[h].y;
-        // sum over the token's 4 lanes: xor 2 keeps heads 4 b1 .., xor 1 keeps
-        // heads 4 b1 + 2 b0 .. = 2q, 2q+1
-        const bool b1 = q >> 1, b0 = q & 1;
-        float x[4];
+        for (int n = 0; n < 2; ++n) {
+            const float2 f = lds64<kUp>(uo[4 + n]);
+            w1[2 * n] = w2[n] * f.x;
+            w1[2 * n + 1] = w2[n] * f.y;
+        }
 #pragma unroll
-        for (int h = 0; h < 4; ++h)
-            x[h] = (b1 ? acc[4 + h] : acc[h]) + __shfl_xor_sync(full, b1 ? acc[h] : acc[4 + h], 2);
-        float y[2];
+        for (int m = 0; m < 4; ++m) {
+            const float2 f = lds64<kUp>(uo[m]);
+            wl[2 * m] = w1[m] * f.x;
+            wl[2 * m + 1] = w1[m] * f.y;
+        }
+        float z;   // head s of this lane's token, summed over the token's 8 lanes
+        if (T == 1) {
+            float2 kk[8];   // (w cos phi, w sin phi) of the block's leaves
 #pragma unroll
-        for (int h = 0; h < 2; ++h) y[h] = (b0 ? x[2 + h] : x[h]) + __shfl_xor_sync(full, b0 ? x[h] : x[2 + h], 1);
-        *(float2*)(pbuf + t * kGQ2 + 2 * q) = (rb & 0x8000u) ? make_float2(-INFINITY, -INFINITY)
-                                                            : make_float2(y[0], y[1]);
+            for (int j = 0; j < 8; ++j) {
+                const float2 f = lds64(lo[j]);
+                kk[j] = make_float2(wl[j] * f.x, wl[j] * f.y);
+            }
+            // slot i of lane s' belongs to lane s' ^ i: each slot pair's sums go
+            // straight to their lanes (a rolled loop keeps the row loads of one
+            // slot pair in flight at a time)
+            z = 0.f;
+#pragma unroll 1
+            for (int hp = 0; hp < 4; ++hp) {   // (q[2j'], q[2j'+1]) of slots 2 hp, 2 hp + 1
+                const uint32_t qr = qb + 128u * hp;
+                float2 ua, uc;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float4 Q;
+                    switch (j) {
+                    case 0: Q = lds128<0>(qr); break;
+                    case 1: Q = lds128<512>(qr); break;
+                    case 2: Q = lds128<1024>(qr); break;
+                    case 3: Q = lds128<1536>(qr); break;
+                    case 4: Q = lds128<2048>(qr); break;
+                    case 5: Q = lds128<2560>(qr); break;
+                    case 6: Q = lds128<3072>(qr); break;
+                    default: Q = lds128<3584>(qr); break;
+                    }
+                    const float2 qa = make_float2(Q.x, Q.y), qc = make_float2(Q.z, Q.w);
+                    ua = j == 0 ? __fmul2_rn(qa, kk[j]) : __ffma2_rn(qa, kk[j], ua);
+                    uc = j == 0 ? __fmul2_rn(qc, kk[j]) : __ffma2_rn(qc, kk[j], uc);
+                }
+                z += __shfl_xor_sync(full, ua.x + ua.y, 2 * hp);
+                z += __shfl_xor_sync(full, uc.x + uc.y, 2 * hp + 1);
+            }
+        } else {
+            float2 acc[4];   // slot pairs (0,1), (2,3), (4,5), (6,7)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float4 F, G;
+                switch (j) {   // leaf j's slab is 4 KB on; the second table 128 bytes on
+                case 0: F = lds128<L::kFold>(lo[j]); G = lds128<L::kFold + L::kFold2>(lo[j]); break;
+                case 1: F = lds128<L::kFold + 4096>(lo[j]); G = lds128<L::kFold + 4096 + L::kFold2>(lo[j]); break;
+                case 2: F = lds128<L::kFold + 8192>(lo[j]); G = lds128<L::kFold + 8192 + L::kFold2>(lo[j]); break;
+                case 3: F = lds128<L::kFold + 12288>(lo[j]); G = lds128<L::kFold + 12288 + L::kFold2>(lo[j]); break;
+                case 4: F = lds128<L::kFold + 16384>(lo[j]); G = lds128<L::kFold + 16384 + L::kFold2>(lo[j]); break;
+                case 5: F = lds128<L::kFold + 20480>(lo[j]); G = lds128<L::kFold + 20480 + L::kFold2>(lo[j]); break;
+                case 6: F = lds128<L::kFold + 24576>(lo[j]); G = lds128<L::kFold + 24576 + L::kFold2>(lo[j]); break;
+                default: F = lds128<L::kFold + 28672>(lo[j]); G = lds128<L::kFold + 28672 + L::kFold2>(lo[j]); break;
+                }
+                const float2 ww = make_float2(wl[j], wl[j]);
+                acc[0] = j == 0 ? __fmul2_rn(ww, make_float2(F.x, F.y)) : __ffma2_rn(ww, make_float2(F.x, F.y), acc[0]);
+                acc[1] = j == 0 ? __fmul2_rn(ww, make_float2(F.z, F.w)) : __ffma2_rn(ww, make_float2(F.z, F.w), acc[1]);
+                acc[2] = j == 0 ? __fmul2_rn(ww, make_float2(G.x, G.y)) : __ffma2_rn(ww, make_float2(G.x, G.y), acc[2]);
+                acc[3] = j == 0 ? __fmul2_rn(ww, make_float2(G.z, G.w)) : __ffma2_rn(ww, make_float2(G.z, G.w), acc[3]);
+            }
+            // reduce-scatter: slot i pairs with slot i + 4 (xor 4), i + 2 (xor 2), i + 1
+            const float x0 = acc[0].x + __shfl_xor_sync(full, acc[2].x, 4);
+            const float x1 = acc[0].y + __shfl_xor_sync(full, acc[2].y, 4);
+            const float x2 = acc[1].x + __shfl_xor_sync(full, acc[3].x, 4);
+            const float x3 = acc[1].y + __shfl_xor_sync(full, acc[3].y, 4);
+            const float y0 = x0 + __shfl_xor_sync(full, x2, 2), y1 = x1 + __shfl_xor_sync(full, x3, 2);
+            z = y0 + __shfl_xor_sync(full, y1, 1);
+        }
+        lg[0] = lg[1];
+        lg[1] = lg[2];
+        lg[2] = lg[3];
+        lg[3] = (rb & 0x8000u) ? -INFINITY : z;
     }
 }
 
@@ -889,31 +884,25 @@ __device__ __forceinline__ void page_logits_mq(const uint8_t* pg, const uint8_t*
 // pair's first / second query sees (the second sees one more token; 0 when
 // the launch has one query).  A head that has seen no token yet keeps an
 // empty state (max -inf, sum 0).
-__device__ __forceinline__ void process_page_mq(const uint8_t* pg, int tier, int valid0, int valid1, const uint8_t* smem,
-                                                float* pbuf, int lane, const uint32_t (&fl)[8], WarpState& st)
+__device__ __forceinline__ void process_page_pair(const uint8_t* pg, int tier, int valid0, int valid1, float* pbuf,
+                                                  int lane, WarpState& st)
 {
     const unsigned full = 0xffffffffu;
-    const int k = lane >> 3, hh = lane & 7;   // softmax: head hh, tokens 4 pass + k
-    if (lane == 0) {
-        ((int*)pbuf)[16 * kGQ2 + kGQ2] = valid0;
-        ((int*)pbuf)[16 * kGQ2 + kGQ2 + 1] = valid1;
-    }
-    if (tier == 1) page_logits_mq<1>(pg, smem, pbuf, lane, fl);
-    else if (tier == 2) page_logits_mq<2>(pg, smem, pbuf, lane, fl);
-    else page_logits_mq<3>(pg, smem, pbuf, lane, fl);
-    __syncwarp();
-    const int valid = ((const int*)pbuf)[16 * kGQ2 + kGQ2 + (hh >> 2)];
-    const int vmax = max(((const int*)pbuf)[16 * kGQ2 + kGQ2], ((const int*)pbuf)[16 * kGQ2 + kGQ2 + 1]);
+    const int k = lane >> 3, s = lane & 7;   // head s, tokens 4 pass + k
     float lg[4];
+    if (tier == 1) page_logits_pair<1>(pg, lane, lg);
+    else if (tier == 2) page_logits_pair<2>(pg, lane, lg);
+    else page_logits_pair<3>(pg, lane, lg);
+    const int valid = s < 4 ? valid0 : valid1, vmax = max(valid0, valid1);
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass)
-        lg[pass] = pass * 4 + k < valid ? pbuf[(pass * 4 + k) * kGQ2 + hh] : -INFINITY;
-    __syncwarp();
+        if (pass * 4 + k >= valid) lg[pass] = -INFINITY;
     float pm = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
     pm = fmaxf(pm, __shfl_xor_sync(full, pm, 8));
     pm = fmaxf(pm, __shfl_xor_sync(full, pm, 16));
     const float m_new = fmaxf(st.m, pm);
-    const float alpha = m_new == -INFINITY ? 1.f : fast_exp2(st.m - m_new);
+    const float m_ref = m_new == -INFINITY ? 0.f : m_new;
+    const float alpha = fast_exp2(st.m - m_ref);
     st.m = m_new;
     const __half* vs = (const __half*)(pg + 2 * kP);
     float wv[4];
@@ -938,12 +927,12 @@ __device__ __forceinline__ void process_page_mq(const uint8_t* pg, int tier, int
     float psum = 0.f;
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
-        const float pv = lg[pass] == -INFINITY ? 0.f : fast_exp2(lg[pass] - m_new);
+        const float pv = fast_exp2(lg[pass] - m_ref);
         psum += pv;
-        pbuf[(pass * 4 + k) * kGQ2 + hh] = pv * wv[pass];
+        pbuf[(pass * 4 + k) * kGQ2 + s] = pv * wv[pass];
     }
     st.l = st.l * alpha + psum;
-    if (lane < kGQ2) pbuf[16 * kGQ2 + hh] = alpha_acc;
+    if (lane < kGQ2) pbuf[16 * kGQ2 + s] = alpha_acc;
     __syncwarp();
     page_values<kGQ2>(pg, tier, pbuf, lane, alpha_acc, st);
     __syncwarp();
@@ -968,18 +957,15 @@ __global__ void __launch_bounds__(Layout<NQ>::kWarps * 32, 1) decode_kernel(Deco
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const unsigned full = 0xffffffffu;
 
-    // Zero point of the layout: shared address 0 for one query (absolute
-    // offsets, the dynamic block must start below the first region), the
-    // dynamic block for a pair.
+    // Zero point of the layout: shared address 0 (absolute offsets; the
+    // dynamic block must start below the first region).
     const uint32_t sbase = smem_u32(smem);
-    if constexpr (NQ == 1) {
-        if (sbase > Layout<1>::kUpT2) {   // cannot happen with <= 8 KB of reserved shared memory
-            if (tid == 0) report(p.status, SPHKV_ERR_DEVICE);
-            return;
-        }
+    if (sbase > L::kUpT2) {   // cannot happen with <= 8 KB of reserved shared memory
+        if (tid == 0) report(p.status, SPHKV_ERR_DEVICE);
+        return;
     }
-    uint8_t* const Z = NQ == 1 ? smem - sbase : smem;
-    const uint32_t zs = NQ == 1 ? 0u : sbase;
+    uint8_t* const Z = smem - sbase;
+    constexpr uint32_t zs = 0;
 
     // cos/sin tables: leaf grid c*2pi/2^b_leaf, upper grid c*(pi/2)/(2^b_up-1)
     for (int e = tid; e < 2 * 256 + 64 + 16; e += kThreads) {
@@ -994,18 +980,13 @@ __global__ void __launch_bounds__(Layout<NQ>::kWarps * 32, 1) decode_kernel(Deco
             off = L::kUpT2 + (e - 512) * 128;
         } else {
             a = 0.5 * (e - 576) / 15;
-            off = L::kUpT3 + (e - 576) * 128;
+            off = L::kUpT3 + (e - 576) * 256;
         }
         double sn, cs;
         sincospi(a, &sn, &cs);
         const float2 v = make_float2((float)cs, (float)sn);
         for (int r = 0; r < 16; ++r) ((float2*)(Z + off))[r] = v;
     }
-    // pairs: per-lane offsets of leaf i of subtree 2 (lane & 3) + ((lane >> 2)
-    // & 1) in the query arrays
-    uint32_t fl[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) fl[i] = (144u * (uint32_t)(2 * (lane & 3) + ((lane >> 2) & 1))) ^ (16u * i);
     uint8_t* stage = Z + L::kStage + w * kS * kStageBytes;
     float* pbuf = (float*)(Z + L::kPbuf) + w * L::kPbufFloats;
     const uint32_t bar0 = zs + L::kBar + w * kS * 8;
@@ -1054,8 +1035,10 @@ __global__ void __launch_bounds__(Layout<NQ>::kWarps * 32, 1) decode_kernel(Deco
         }
         // One query: this lane's query slice in registers, q[16s .. 16s+15] of
         // the 4 heads times the logit scale, in the lane's slot order (see
-        // page_logits), and the unit's query-folded T2/T3 leaf table (the
-        // previous segment ended with a barrier, so no warp still reads it).
+        // page_logits).  Both: the unit's query-folded T2/T3 leaf tables, and
+        // for a pair the T1 query rows (the previous segment ended with a
+        // barrier, so no warp still reads them).  A pair launch with one query
+        // (npair = 1) has heads 4-7 empty: their query is 0.
         float2 qp[kG][8];
         if constexpr (NQ == 1) {
             const int s = lane & 7, b2 = (s >> 2) & 1, b1 = (s >> 1) & 1;
@@ -1070,6 +1053,8 @@ __global__ void __launch_bounds__(Layout<NQ>::kWarps * 32, 1) decode_kernel(Deco
                     qp[i][2 * k + 1] = make_float2(v.z * kLogitScale, v.w * kLogitScale);
                 }
             }
+        }
+        if constexpr (NQ == 1) {
             for (int e = tid; e < 16 * kLeaves; e += kThreads) {
                 const int code = e >> 6, j = e & 63, sj = j >> 3, ij = j & 7;
                 const int c2 = (sj >> 2) & 1, c1 = (sj >> 1) & 1;   // slot order of the lanes owning subtree sj
@@ -1081,22 +1066,37 @@ __global__ void __launch_bounds__(Layout<NQ>::kWarps * 32, 1) decode_kernel(Deco
                     const float* qh = p.q + out_row(p, b, g, h) * kD;
                     v[k] = fmaf(qh[2 * j + 1], cs.y, qh[2 * j] * cs.x) * kLogitScale;
                 }
-                *(float4*)(Z + L::kFold + ((uint32_t)code << 11) + 144 * sj + 16 * ij) =
+                *(float4*)(Z + L::kFold + (ij << 12) + ((uint32_t)code << 8) + (sj << 4)) =
                     make_float4(v[0], v[1], v[2], v[3]);
             }
-        } else {   // the pair's query rows (the previous segment ended with a barrier)
+        } else {
+            // folded tables: table tb holds slots 4 tb .. 4 tb + 3 (head (4 tb + k) ^ s)
+            for (int e = tid; e < 2 * 16 * kLeaves; e += kThreads) {
+                const int tb = e >> 10, code = (e >> 6) & 15, j = e & 63, sj = j >> 3, ij = j & 7;
+                const float2 cs = *(const float2*)(Z + L::kT1 + 16 * code * 256);
+                float v[kG];
+#pragma unroll
+                for (int k = 0; k < kG; ++k) {
+                    const int h = (4 * tb + k) ^ sj;
+                    const float* qh = p.q + out_row(p, b, g, (h >> 2) < p.npair ? h : 0) * kD;
+                    v[k] = (h >> 2) < p.npair ? fmaf(qh[2 * j + 1], cs.y, qh[2 * j] * cs.x) * kLogitScale : 0.f;
+                }
+                *(float4*)(Z + L::kFold + (ij << 12) + ((uint32_t)code << 8) + tb * L::kFold2 + (sj << 4)) =
+                    make_float4(v[0], v[1], v[2], v[3]);
+            }
+            // T1 query rows: (q[2j], q[2j+1]) of slots 2 hp, 2 hp + 1
             for (int e = tid; e < 4 * kLeaves; e += kThreads) {
-                const int a = e >> 6, j = e & 63, sj = j >> 3, ij = j & 7;
+                const int hp = e >> 6, j = e & 63, sj = j >> 3, ij = j & 7;
                 float v[4];
 #pragma unroll
-                for (int hp = 0; hp < 2; ++hp) {
-                    const int hh = 2 * a + hp;
-                    const bool live = (hh >> 2) < p.npair;
-                    const float* qh = p.q + out_row(p, b, g, live ? hh : 0) * kD + 2 * j;
-                    v[2 * hp] = live ? qh[0] : 0.f;
-                    v[2 * hp + 1] = live ? qh[1] : 0.f;
+                for (int u = 0; u < 2; ++u) {
+                    const int h = (2 * hp + u) ^ sj;
+                    const bool live = (h >> 2) < p.npair;
+                    const float* qh = p.q + out_row(p, b, g, live ? h : 0) * kD + 2 * j;
+                    v[2 * u] = live ? qh[0] * kLogitScale : 0.f;
+                    v[2 * u + 1] = live ? qh[1] * kLogitScale : 0.f;
                 }
-                *(float4*)(Z + L::kQ + 1024 * a + ((144 * sj) ^ (16 * ij))) = make_float4(v[0], v[1], v[2], v[3]);
+                *(float4*)(Z + L::kQ + 512 * ij + 128 * hp + 16 * sj) = make_float4(v[0], v[1], v[2], v[3]);
             }
         }
         __syncthreads();
@@ -1245,7 +1245,7 @@ __global__ void __launch_bounds__(Layout<NQ>::kWarps * 32, 1) decode_kernel(Deco
                 process_page(pg, t, valid, pbuf, lane, qp, st);
             } else {
                 const int v0 = max(0, min(kP, len - lpq[0] * kP)), v1 = max(0, min(kP, len2 - lpq[0] * kP));
-                process_page_mq(pg, t, v0, v1, smem, pbuf, lane, fl, st);
+                process_page_pair(pg, t, v0, v1, pbuf, lane, st);
             }
 #pragma unroll
             for (int i = 0; i < kS - 1; ++i) {

@@ -211,9 +211,10 @@ def test_multi_query_decode(n_q):
         assert np.array_equal(o1, out[:, 0]) and np.array_equal(l1, lse[:, 0])
 
 
-def test_multi_query_full_size_sampled():
+def test_multi_query_full_size_every_unit():
     """Two query tokens per sequence at the 32k workload's full size, on the
-    launch path bench.py --n-q 2 times; sampled units against the oracle."""
+    launch path bench.py --n-q 2 times (one launch of the pair kernel): every
+    (query, sequence, kv head) unit against the oracle."""
     torch = _torch()
     w = W.make("llama32k")
     cache = gpu_cache(w)
@@ -222,11 +223,13 @@ def test_multi_query_full_size_sampled():
     out, lse = cache.decode_mq(to_torch(q, torch.float32))
     cache.check()
     out, lse = out.cpu().numpy(), lse.cpu().numpy()
-    for b, g in [(0, 0), (5, 7)]:
-        for i in range(2):
-            lens = np.maximum(w.seq_lens - (1 - i), 0)
-            ro, rl = oracle_unit(w, b, g, q[:, i], lens=lens)
-            assert_close(out[b, i, 4 * g:4 * g + 4], lse[b, i, 4 * g:4 * g + 4], ro, rl, f"query {i} unit {(b, g)}")
+    ref = oracle_full_cache(w)
+    units = [(b, g) for b in range(w.B) for g in range(w.H_kv)]
+    ro, rl = oracle.multi_query_attention(ref, q, units, 2)
+    for i in range(2):
+        for k, (b, g) in enumerate(units):
+            assert_close(out[b, i, 4 * g:4 * g + 4], lse[b, i, 4 * g:4 * g + 4], ro[i, k], rl[i, k],
+                         f"query {i} unit {(b, g)}")
 
 
 def test_physical_permutation_is_bit_identical():
