@@ -11,11 +11,22 @@
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include "../../include/sphkv.h"
 
 namespace sphkv {
+
+// A named NVTX range around one C-ABI call, so that timeline tools (nsys, ncu's
+// range filters) can attribute the call's launches; without a tool attached
+// it costs a load and a branch.
+struct CallRange {
+    explicit CallRange(const char* name) { nvtxRangePushA(name); }
+    ~CallRange() { nvtxRangePop(); }
+    CallRange(const CallRange&) = delete;
+    CallRange& operator=(const CallRange&) = delete;
+};
 
 constexpr int kD = SPHKV_HEAD_DIM;      // 128
 constexpr int kP = SPHKV_PAGE_TOKENS;   // 16

@@ -1535,6 +1535,7 @@ extern "C" sphkv_status sphkv_decode_attention(const sphkv_cache* c, int32_t H_q
                                                size_t ws_bytes, int32_t* status_dev, void* stream)
 {
     const char* fn = "sphkv_decode_attention";
+    const CallRange range(fn);
     DecodeParams p;
     sphkv_status st = fill_params(fn, c, H_q, q, out, lse, status_dev, p);
     if (st != SPHKV_OK) return st;
@@ -1569,6 +1570,7 @@ extern "C" sphkv_status sphkv_decode_attention_mq(const sphkv_cache* c, int32_t 
                                                   int32_t* status_dev, void* stream)
 {
     const char* fn = "sphkv_decode_attention_mq";
+    const CallRange range(fn);
     DecodeParams p;
     sphkv_status st = fill_params(fn, c, H_q, q, out, lse, status_dev, p);
     if (st != SPHKV_OK) return st;
@@ -1621,6 +1623,7 @@ extern "C" sphkv_status sphkv_decode_attention_noalloc(const sphkv_cache* c, int
                                                        void* stream)
 {
     const char* fn = "sphkv_decode_attention_noalloc";
+    const CallRange range(fn);
     DecodeParams p;
     sphkv_status st = fill_params(fn, c, H_q, q, out, lse, status_dev, p);
     if (st != SPHKV_OK) return st;

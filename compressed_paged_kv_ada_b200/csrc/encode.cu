@@ -440,6 +440,7 @@ extern "C" sphkv_status sphkv_migrate(const sphkv_cache* from, const sphkv_cache
                                       void* stream)
 {
     const char* fn = "sphkv_migrate";
+    const CallRange range(fn);
     if (!from || !to) {
         sphkv_set_error("%s: null argument", fn);
         return SPHKV_ERR_ARG;
@@ -484,6 +485,7 @@ extern "C" sphkv_status sphkv_encode(const sphkv_cache* c, const void* K, const 
                                      const int32_t* tok_seq, const int32_t* tok_pos, int64_t n_tok,
                                      int32_t* status_dev, void* stream)
 {
+    const CallRange range("sphkv_encode");
     if (!c || (n_tok > 0 && (!K || !V || !tok_seq || !tok_pos))) {
         sphkv_set_error("sphkv_encode: null argument");
         return SPHKV_ERR_ARG;

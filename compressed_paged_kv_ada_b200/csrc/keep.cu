@@ -68,6 +68,7 @@ using namespace sphkv;
 extern "C" sphkv_status sphkv_set_keep(const sphkv_cache* c, const uint8_t* keep, int32_t* status_dev, void* stream)
 {
     const char* fn = "sphkv_set_keep";
+    const CallRange range(fn);
     if (!c || !keep) {
         sphkv_set_error("%s: null argument", fn);
         return SPHKV_ERR_ARG;

@@ -362,6 +362,7 @@ extern "C" sphkv_status sphkv_rdr_assign(const sphkv_cache* c, const float* util
                                          void* workspace, size_t ws_bytes, int32_t* status_dev,
                                          void* stream)
 {
+    const CallRange range("sphkv_rdr_assign");
     return rdr_launch("sphkv_rdr_assign", false, c, utility, eps, budget_bytes, n_sink, n_recent, tiers_out,
                       lambda_out, bytes_out, workspace, ws_bytes, status_dev, stream);
 }
@@ -371,6 +372,7 @@ extern "C" sphkv_status sphkv_rdr_rerun(const sphkv_cache* c, const float* utili
                                         double* lambda_out, int64_t* bytes_out, void* workspace, size_t ws_bytes,
                                         int32_t* status_dev, void* stream)
 {
+    const CallRange range("sphkv_rdr_rerun");
     return rdr_launch("sphkv_rdr_rerun", true, c, utility, eps, budget_bytes, n_sink, n_recent, tiers_io,
                       lambda_out, bytes_out, workspace, ws_bytes, status_dev, stream);
 }
@@ -459,6 +461,7 @@ extern "C" sphkv_status sphkv_build_page_table(const uint8_t* tiers, int64_t n_e
                                                const int32_t* perm2, const int32_t* perm3, int32_t* table,
                                                int64_t* counts_out, int32_t* status_dev, void* stream)
 {
+    const CallRange range("sphkv_build_page_table");
     if (n_entries < 0 || (n_entries > 0 && (!tiers || !table))) {
         sphkv_set_error("sphkv_build_page_table: bad arguments");
         return SPHKV_ERR_ARG;

@@ -44,6 +44,7 @@ extern "C" sphkv_status sphkv_merge_partials(const float* out_parts, const float
                                              int64_t n_rows, float* out, float* lse, void* stream)
 {
     const char* fn = "sphkv_merge_partials";
+    const CallRange range(fn);
     if (n_rows < 0 || n_parts < 1 || n_parts > 4096) {
         sphkv_set_error("%s: need 1 <= n_parts <= 4096 and n_rows >= 0 (got %d, %lld)", fn, n_parts,
                         (long long)n_rows);
