@@ -2,10 +2,13 @@
 
     python -m compressed_paged_kv_ada_b200.build [--force] [--verbose]
 
-It also builds libsphkv_testhooks.so, the same library with decode.cu
-compiled with -DSPHKV_TEST_HOOKS, which only the tests load (they use it to
-make a bounded device wait run out without any fault).  The product library
-is built without the flag.
+It also builds two variants that only the tests load; the product library is
+built without their flags:
+- libsphkv_testhooks.so: decode.cu compiled with -DSPHKV_TEST_HOOKS (the tests
+  use it to make a bounded device wait run out without any fault);
+- libsphkv_debug.so: decode.cu compiled with -DSPHKV_DEBUG (every shared-memory
+  table address checked against its table, a canary past each shorter page
+  copy, and a stream synchronisation after every call).
 
 encode.cu and rdr.cu are compiled with -fmad=false: their fp64 arithmetic must
 not be contracted into fused multiply-adds (codes and tier decisions are
@@ -23,6 +26,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsphkv.so")
 TEST_LIB = os.path.join(HERE, "libsphkv_testhooks.so")
+DEBUG_LIB = os.path.join(HERE, "libsphkv_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -53,11 +57,11 @@ def _link(objs, out):
 def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     newest = max(os.path.getmtime(f) for f in _deps())
-    if (not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest and os.path.exists(TEST_LIB)
-            and os.path.getmtime(TEST_LIB) >= newest):
+    if not force and all(os.path.exists(f) and os.path.getmtime(f) >= newest for f in (LIB, TEST_LIB, DEBUG_LIB)):
         return LIB
     objs = {}
-    for src, extra in list(SOURCES.items()) + [("decode.cu#hooks", ["-DSPHKV_TEST_HOOKS"])]:
+    variants = [("decode.cu#hooks", ["-DSPHKV_TEST_HOOKS"]), ("decode.cu#debug", ["-DSPHKV_DEBUG"])]
+    for src, extra in list(SOURCES.items()) + variants:
         name = src.split("#")[0]
         obj = os.path.join(BUILD, src.replace(".cu", "").replace("#", "_") + ".o")
         cmd = [NVCC, *ARCH, *COMMON, *extra, "-c", os.path.join(CSRC, name), "-o", obj]
@@ -68,6 +72,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         objs[src] = obj
     _link([objs[s] for s in SOURCES], LIB)
     _link([objs[s] for s in SOURCES if s != "decode.cu"] + [objs["decode.cu#hooks"]], TEST_LIB)
+    _link([objs[s] for s in SOURCES if s != "decode.cu"] + [objs["decode.cu#debug"]], DEBUG_LIB)
     return LIB
 
 

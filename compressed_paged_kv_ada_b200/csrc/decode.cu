@@ -131,10 +131,13 @@ constexpr bool layout_ok()
                L::kWarps * L::kStages * kStageBytes;
 }
 static_assert(layout_ok<1>() && layout_ok<2>(), "shared-memory layout");
-static_assert(Layout<1>::kSlice + Layout<1>::kWarps * 4 <= Layout<1>::kFold && Layout<1>::kFold % 32768 == 0 &&
+// word after the slice sums: violations seen by the debug build's checks
+template <int NQ>
+constexpr uint32_t kDbgFlag = Layout<NQ>::kSlice + 4 * Layout<NQ>::kWarps;
+static_assert(Layout<1>::kSlice + Layout<1>::kWarps * 4 + 4 <= Layout<1>::kFold && Layout<1>::kFold % 32768 == 0 &&
                   Layout<1>::kFold + 32768 <= Layout<1>::kT1 && Layout<1>::kT1 + 65536 <= Layout<1>::kStage,
               "one-query regions");
-static_assert(Layout<2>::kSlice + Layout<2>::kWarps * 4 <= Layout<2>::kQ && Layout<2>::kQ % 128 == 0 &&
+static_assert(Layout<2>::kSlice + Layout<2>::kWarps * 4 + 4 <= Layout<2>::kQ && Layout<2>::kQ % 128 == 0 &&
                   Layout<2>::kQ + 4096 <= Layout<2>::kFold && Layout<2>::kFold % 32768 == 0 &&
                   Layout<2>::kFold + 32768 <= Layout<2>::kT1 &&
                   Layout<2>::kT1 + 65536 <= Layout<2>::kStage && Layout<1>::kUpT2 == Layout<2>::kUpT2,
@@ -447,6 +450,48 @@ __device__ __forceinline__ void block_addrs(const uint8_t* codes, int blk, uint3
     }
 }
 
+#ifdef SPHKV_DEBUG
+// Debug builds (-DSPHKV_DEBUG) check every table address a subtree block
+// computes against the table it indexes: the load's address (register plus
+// immediate) must lie inside the table and be aligned to the load's width.  A
+// bad address sets the CTA's flag word (reported as SPHKV_ERR_DEVICE at the
+// end of the segment) and is replaced by one inside the table, so the checked
+// build never reads outside its tables either.
+template <int NQ>
+__device__ __forceinline__ void dbg_fix(uint32_t& a, uint32_t imm, uint32_t base, uint32_t size, uint32_t align)
+{
+    const uint32_t x = a + imm;
+    if (x < base || x + align > base + size || (x & (align - 1))) {
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(kDbgFlag<NQ>), "r"(1u) : "memory");
+        a = base - imm;
+    }
+}
+
+// lo: leaf lookups (T1 rows, or the folded table(s) with leaf j's slab at
+// 4096 j and, for a pair, the second table 128 bytes on); uo: upper lookups.
+template <int NQ, int T>
+__device__ __forceinline__ void dbg_check_block(uint32_t (&lo)[8], uint32_t (&uo)[8])
+{
+    using L = Layout<NQ>;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        if (T == 1) {
+            dbg_fix<NQ>(lo[j], 0, L::kT1, 65536, 8);
+            if (lo[j] & 128u) {   // a leaf address must stay in the leaf half of its row
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(kDbgFlag<NQ>), "r"(1u) : "memory");
+                lo[j] &= ~128u;
+            }
+            dbg_fix<NQ>(uo[j], 128, L::kT1, 65536, 8);
+        } else {
+            dbg_fix<NQ>(lo[j], L::kFold + 4096 * j, L::kFold + 4096 * j, 4096, 16);
+            if (NQ == 2) dbg_fix<NQ>(lo[j], L::kFold + 4096 * j + 128, L::kFold + 4096 * j, 4096, 16);
+            if (T == 2) dbg_fix<NQ>(uo[j], 0, L::kUpT2, 8192, 8);
+            else dbg_fix<NQ>(uo[j], L::kUpT3, L::kUpT3, 4096, 8);
+        }
+    }
+}
+#endif
+
 // Logits of the 16 tokens of one page of tier T staged at `pg`, in the log2
 // domain: lane (k4, s) ends with lg[pass] = the logit of token 4 pass + k4 for
 // head 2 b2 + b1 (s = 4 b2 + 2 b1 + b0).  Eight lanes per token, four tokens per
@@ -488,6 +533,9 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, int lane, const f
         const int t = pass * 4 + (lane >> 3);
         uint32_t lo[8], uo[8];
         block_addrs<T>(codes, pass * 32 + lane, rep1, repU, fb, lo, uo);
+#ifdef SPHKV_DEBUG
+        dbg_check_block<1, T>(lo, uo);
+#endif
         // ancestors: top node s/2 (level 4), 4 + s/4 (level 5), 6 (root)
         const uint32_t o4 = __shfl_sync(full, uo[7], grp + (s >> 1));
         const uint32_t o5 = __shfl_sync(full, uo[7], grp + 4 + (s >> 2));
@@ -782,6 +830,9 @@ __device__ __forceinline__ void page_logits_pair(const uint8_t* pg, int lane, fl
         const int t = pass * 4 + (lane >> 3);
         uint32_t lo[8], uo[8];
         block_addrs<T>(codes, pass * 32 + lane, rep1, repU, fb, lo, uo);
+#ifdef SPHKV_DEBUG
+        dbg_check_block<2, T>(lo, uo);
+#endif
         const uint32_t o4 = __shfl_sync(full, uo[7], grp + (s >> 1));
         const uint32_t o5 = __shfl_sync(full, uo[7], grp + 4 + (s >> 2));
         const uint32_t o6 = __shfl_sync(full, uo[7], grp + 6);
@@ -995,6 +1046,9 @@ __global__ void __launch_bounds__(Layout<NQ>::kWarps * 32, 1) decode_kernel(Deco
         for (int i = 0; i < kS; ++i) mbar_init(bar0 + 8 * i, 1);
         fence_barrier_init();
     }
+#ifdef SPHKV_DEBUG
+    if (tid == 0) *(volatile uint32_t*)(Z + kDbgFlag<NQ>) = 0u;
+#endif
     __syncthreads();
 
     asm volatile("griddepcontrol.wait;" ::: "memory");   // plan_kernel's results are visible
@@ -1183,6 +1237,12 @@ __global__ void __launch_bounds__(Layout<NQ>::kWarps * 32, 1) decode_kernel(Deco
         auto issue = [&](int stg, int32_t e) {
             if (lane == 0) {
                 const uint32_t bytes = (uint32_t)page_bytes_of(entry_tier(e));
+#ifdef SPHKV_DEBUG
+                // a canary in the stage's last word, past a shorter page: the
+                // copy must not reach it
+                if (bytes + 4 <= (uint32_t)kStageBytes)
+                    *(volatile uint32_t*)(stage + stg * kStageBytes + kStageBytes - 4) = 0x5AFEC0DEu;
+#endif
                 fence_proxy_async();
                 mbar_expect_tx(bar0 + 8 * stg, bytes);
                 bulk_g2s(smem_u32(stage + stg * kStageBytes), page_src(e), bytes, bar0 + 8 * stg);
@@ -1239,6 +1299,11 @@ __global__ void __launch_bounds__(Layout<NQ>::kWarps * 32, 1) decode_kernel(Deco
                 break;
             }
             const uint8_t* pg = stage + cur * kStageBytes;
+#ifdef SPHKV_DEBUG
+            if (lane == 0 && page_bytes_of(entry_tier(eq[0])) + 4 <= kStageBytes &&
+                *(volatile const uint32_t*)(pg + kStageBytes - 4) != 0x5AFEC0DEu)
+                *(volatile uint32_t*)(Z + kDbgFlag<NQ>) = 1u;
+#endif
             const int t = entry_tier(eq[0]);
             if constexpr (NQ == 1) {
                 const int valid = min(kP, len - lpq[0] * kP);
@@ -1323,6 +1388,12 @@ __global__ void __launch_bounds__(Layout<NQ>::kWarps * 32, 1) decode_kernel(Deco
             }
         }
         __syncthreads();   // scratch free before the next segment's copies
+#ifdef SPHKV_DEBUG
+        if (tid == 0 && *(volatile uint32_t*)(Z + kDbgFlag<NQ>)) {
+            report(p.status, SPHKV_ERR_DEVICE);
+            *(volatile uint32_t*)(Z + kDbgFlag<NQ>) = 0u;
+        }
+#endif
         x = seg_end;
         if (failed) break;
     }
@@ -1506,9 +1577,17 @@ sphkv_status ensure_smem(const char* fn)
     return SPHKV_OK;
 }
 
-sphkv_status launched(const char* fn)
+// After the launches of a call: a launch error is reported.  Debug builds also
+// wait for the call's kernels (the only place the library synchronises) so
+// that an execution error surfaces at the call that caused it.
+sphkv_status launched(const char* fn, void* stream)
 {
-    const cudaError_t err = cudaGetLastError();
+    cudaError_t err = cudaGetLastError();
+#ifdef SPHKV_DEBUG
+    if (err == cudaSuccess) err = cudaStreamSynchronize((cudaStream_t)stream);
+#else
+    (void)stream;
+#endif
     if (err != cudaSuccess) {
         sphkv_set_error("%s: launch failed: %s", fn, cudaGetErrorString(err));
         return SPHKV_ERR_DEVICE;
@@ -1553,7 +1632,7 @@ extern "C" sphkv_status sphkv_decode_attention(const sphkv_cache* c, int32_t H_q
     p.partial = (float*)((uint8_t*)workspace + part_off);
     if ((st = ensure_smem(fn)) != SPHKV_OK) return st;
     launch_decode<1>(p, (cudaStream_t)stream);
-    return launched(fn);
+    return launched(fn, stream);
 }
 
 extern "C" size_t sphkv_decode_mq_workspace_bytes(int32_t B, int32_t H_q, int32_t H_kv, int64_t total_pages,
@@ -1600,7 +1679,7 @@ extern "C" sphkv_status sphkv_decode_attention_mq(const sphkv_cache* c, int32_t 
         p.len_shift = n_q - q0 - p.npair;
         if (p.npair == 2) launch_decode<2>(p, (cudaStream_t)stream);
         else launch_decode<1>(p, (cudaStream_t)stream);
-        if ((st = launched(fn)) != SPHKV_OK) return st;
+        if ((st = launched(fn, stream)) != SPHKV_OK) return st;
     }
     return SPHKV_OK;
 }
@@ -1651,5 +1730,5 @@ extern "C" sphkv_status sphkv_decode_attention_noalloc(const sphkv_cache* c, int
     p.unit_start = (int32_t*)scratch;
     p.partial = (float*)((uint8_t*)scratch + part_off);
     launch_decode<1>(p, (cudaStream_t)stream);
-    return launched(fn);
+    return launched(fn, stream);
 }
