@@ -124,6 +124,23 @@ def served_units(w, n_q: int = 1, lens=None) -> int:
     return int(sum(np.maximum(lens - (n_q - 1 - i), 0).sum() for i in range(n_q))) * w.H_q
 
 
+def kept_units(w, n_q: int = 1) -> int:
+    """Token-heads of kept tokens only (pages not dropped) that one step
+    serves: the other reading of the metric, which leaves dropped work out."""
+    lens = np.asarray(w.seq_lens, np.int64)
+    po = w.page_offsets
+    G = w.H_q // w.H_kv
+    total = 0
+    for i in range(n_q):
+        for b in range(w.B):
+            n = max(int(lens[b]) - (n_q - 1 - i), 0)
+            npg = (n + 15) // 16
+            valid = np.minimum(16, n - 16 * np.arange(npg))
+            for g in range(w.H_kv):
+                total += int(valid[w.tiers[g, po[b]:po[b] + npg] != 0].sum()) * G
+    return total
+
+
 def algorithmic_bytes(w, lens=None, tiers=None) -> int:
     """Exact bytes the decode must move for one step: the bits of every kept
     token, one page-table entry per token-holding page, q, out and lse."""
@@ -496,6 +513,7 @@ def run_gpu(args):
                        "l2": ("the compressed cache (under 1 MB) fits in L2 and stays there between steps; no flush"
                               if fits_l2 else "compressed cache per step larger than L2 (126 MB); no flush"),
                        "algorithmic_bytes_per_step": algo,
+                       "kept_token_heads_per_s": kept_units(w, n_q) * world / (t_max / 1e3),
                        "hbm_gbs_per_gpu": roof["achieved"], "hbm_frac_of_8tbs": roof["achieved"] / 8000.0},
             "roofline": roof,
             "cpu_baseline": cb,
