@@ -701,12 +701,8 @@ __device__ __forceinline__ void page_values(const uint8_t* pg, int tier, const f
         const int ch = 16 * (g ^ (2 * c));
         const uint4 XY = *(const uint4*)(vrow + c * 128 + ch);
         const uint4 ZW = *(const uint4*)(vrow + (c + 4) * 128 + ch);
-        const uint2 X = make_uint2(XY.x, XY.y), Y = make_uint2(XY.z, XY.w);
-        const uint2 Z = make_uint2(ZW.x, ZW.y), W = make_uint2(ZW.z, ZW.w);
-        const uint32_t xs[2] = {X.x ^ 0x88888888u, X.y ^ 0x88888888u};
-        const uint32_t ys[2] = {Y.x ^ 0x88888888u, Y.y ^ 0x88888888u};
-        const uint32_t zs[2] = {Z.x ^ 0x88888888u, Z.y ^ 0x88888888u};
-        const uint32_t ws[2] = {W.x ^ 0x88888888u, W.y ^ 0x88888888u};
+        const uint32_t xs[2] = {XY.x, XY.y}, ys[2] = {XY.z, XY.w};
+        const uint32_t zs[2] = {ZW.x, ZW.y}, ws[2] = {ZW.z, ZW.w};
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
             const int wi = m >> 2, b = m & 3;   // byte m: low nibble h = 0, high nibble h = 1
@@ -714,12 +710,14 @@ __device__ __forceinline__ void page_values(const uint8_t* pg, int tier, const f
             const uint32_t xy = __byte_perm(xs[wi], ys[wi], sel);
             const uint32_t zw = __byte_perm(zs[wi], ws[wi], sel);
             // low nibble: f16 1024 + u; high nibble in place: f16 1024 + 16 u,
-            // scaled by 1/16 in the bias step (all exact in f16)
+            // scaled by 1/16 in the bias step (all exact in f16).  u = v + 8
+            // (offset binary) is the nibble's top bit flipped, folded with the
+            // mask and the exponent bits into one (x & mask) ^ pattern.
             uint32_t a[4];
-            a[0] = (xy & 0x000F000Fu) | 0x64006400u;
-            a[1] = (xy & 0x00F000F0u) | 0x64006400u;
-            a[2] = (zw & 0x000F000Fu) | 0x64006400u;
-            a[3] = (zw & 0x00F000F0u) | 0x64006400u;
+            a[0] = (xy & 0x000F000Fu) ^ 0x64086408u;
+            a[1] = (xy & 0x00F000F0u) ^ 0x64806480u;
+            a[2] = (zw & 0x000F000Fu) ^ 0x64086408u;
+            a[3] = (zw & 0x00F000F0u) ^ 0x64806480u;
 #pragma unroll
             for (int i = 0; i < 4; i += 2) {
                 const __half2 lo = __hadd2(*(const __half2*)&a[i], bias);
