@@ -507,7 +507,8 @@ __device__ __forceinline__ void dbg_check_block(uint32_t (&lo)[8], uint32_t (&uo
 // head.  T1 leaves: (cos, sin) from the table times the path weight, then one
 // packed multiply-add per head with the lane's query slice (q[16s..16s+15] of
 // the 4 heads, logit scale included) in registers.  T2/T3 leaves: one 16-byte
-// lookup of the unit's query-folded table, two packed multiply-adds.  Both
+// lookup of the unit's query-folded table, two packed multiply-adds
+// (even and odd leaves in separate chains, added at the end).  Both
 // keep the heads in the lane's slot order (slot i holds head ((i >> 1) ^ b2)
 // * 2 + ((i & 1) ^ b1) for s = 4 b2 + 2 b1 + b0), which makes the 8-lane sum
 // a select-free reduce-scatter that leaves head 2 b2 + b1 in lanes b0 = 0, 1.
@@ -579,7 +580,7 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, int lane, const f
 #pragma unroll
             for (int i = 0; i < kG; ++i) a[i] = acc[i].x + acc[i].y;
         } else {
-            float2 acc01, acc23;
+            float2 acc01[2], acc23[2];   // even and odd leaves: two chains per head pair
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 float4 F;
@@ -594,13 +595,15 @@ __device__ __forceinline__ void page_logits(const uint8_t* pg, int lane, const f
                 default: F = lds128<L::kFold + 28672>(lo[j]); break;
                 }
                 const float2 ww = make_float2(wl[j], wl[j]);
-                acc01 = j == 0 ? __fmul2_rn(ww, make_float2(F.x, F.y)) : __ffma2_rn(ww, make_float2(F.x, F.y), acc01);
-                acc23 = j == 0 ? __fmul2_rn(ww, make_float2(F.z, F.w)) : __ffma2_rn(ww, make_float2(F.z, F.w), acc23);
+                const int e = j & 1;
+                acc01[e] = j < 2 ? __fmul2_rn(ww, make_float2(F.x, F.y)) : __ffma2_rn(ww, make_float2(F.x, F.y), acc01[e]);
+                acc23[e] = j < 2 ? __fmul2_rn(ww, make_float2(F.z, F.w)) : __ffma2_rn(ww, make_float2(F.z, F.w), acc23[e]);
             }
-            a[0] = acc01.x;
-            a[1] = acc01.y;
-            a[2] = acc23.x;
-            a[3] = acc23.y;
+            const float2 s01 = __fadd2_rn(acc01[0], acc01[1]), s23 = __fadd2_rn(acc23[0], acc23[1]);
+            a[0] = s01.x;
+            a[1] = s01.y;
+            a[2] = s23.x;
+            a[3] = s23.y;
         }
         const float r0 = a[0] + __shfl_xor_sync(full, a[2], 4);
         const float r1 = a[1] + __shfl_xor_sync(full, a[3], 4);
