@@ -16,30 +16,34 @@
 // are programmatic dependent launches that overlap the previous kernel's
 // tail and wait for its results):
 //   plan   -- 1 CTA: unit_start[u] = pages before unit u = (b, g), u = b*H_kv+g.
-//   decode -- persistent, one 512-thread CTA per SM.  The flattened page range
-//             [0, P) is cut into n_cta equal pieces; a CTA walks the units its
-//             piece overlaps.  Its 16 warps split each unit's pages into
+//   decode -- persistent, one 384-thread CTA (12 warps) per SM.  The flattened
+//             page range [0, P) is cut into n_cta equal pieces; a CTA walks the
+//             units its piece overlaps.  Its warps split each unit's pages into
 //             contiguous ranges of equal tier weight; each warp bulk-copies a
 //             page (cp.async.bulk, mbarrier completion) into a 2-stage ring in
 //             shared memory while it computes the previous one.
-//             Logits, top down: 8 tokens per pass, 4 lanes per token; lane q
-//             owns subtree blocks 2q, 2q+1 (one level-4 node) for all 4 query
-//             heads, so each table lookup serves 4 heads.  The top codes come
-//             by shuffles, and a two-stage butterfly leaves each lane one head.
-//             Cos/sin tables sit in shared memory with 16 lane replicas per
-//             code, so a half warp's 64-bit lookups never share a bank.  T2/T3
-//             leaves (16 and 8 codes) instead index a per-unit table that
-//             already holds q[2j] cos(phi) + q[2j+1] sin(phi) for the 4 heads:
-//             one 16-byte lookup per leaf.  (Packed f32x2 arithmetic in the
-//             upper levels would need {cos,cos} and {sin,sin} pairs, i.e.
-//             16-byte lookups; measured on B200 that doubles shared-memory
-//             traffic and is slower.)
-//             Values: out^T[dims x heads] += V^T[dims x 16 tokens] P^T[16 x 4]
-//             on the tensor cores (mma.sync m16n8k16, f16 operands, fp32
+//             Logits, top down: 4 tokens per pass, 8 lanes per token; lane
+//             (k, s) owns subtree block s (8 leaves, 7 upper nodes) of its
+//             token for every head of the unit, gets the three ancestors' codes
+//             by shuffle, and forms the leaves' path products once for all
+//             heads.  T1 leaves: a (cos, sin) lookup times the path weight,
+//             dotted with the lane's query slice in registers.  T2/T3 leaves:
+//             one 16-byte lookup in a per-unit table that already holds
+//             q[2j] cos(phi) + q[2j+1] sin(phi) for 4 heads.  The tables sit at
+//             absolute shared addresses with lane replicas, a code becomes an
+//             address with one byte permute (8- and 4-bit codes) or a shift
+//             and a masked OR, and the heads are kept in a lane-dependent
+//             order so that the 8-lane sum is a select-free reduce-scatter
+//             leaving each lane one head; the logits stay in registers into
+//             the online softmax.
+//             Values: out^T[dims x heads] += V^T[dims x 16 tokens] P^T on the
+//             tensor cores (mma.sync m16n8k16, f16 operands, fp32
 //             accumulators).  Value codes are exact in f16; the weights
-//             p * vscale * sc are split into f16 hi + lo parts (two MMAs),
-//             keeping ~22 bits.
-//   merge  -- one CTA per unit whose pages were split over several CTAs.
+//             p * vscale * sc are split into f16 hi + lo parts, keeping ~22
+//             bits (one query: both parts in one MMA, columns 0-3 and 4-7; a
+//             pair: two MMAs).
+//   merge  -- one CTA per unit; only units whose pages were split over
+//             several CTAs do any work.
 // decode_kernel<1> serves one query token per sequence (4 query heads per kv
 // head); decode_kernel<2> serves a pair of causal query tokens (8 heads), see
 // "two query tokens per pass" below.
@@ -319,9 +323,9 @@ __device__ inline int32_t cta_bound(int c, int32_t P, int n_cta)
     return (int32_t)(((int64_t)c * P) / n_cta);
 }
 
-// Work of a page by tier, for splitting a CTA's pages among its warps: a T1
-// page takes about 4/3 of the time of a T2 or T3 page; dropped pages are
-// skipped.
+// Work of a page by tier, for splitting a CTA's pages among its warps: 4 for
+// a T1 page, 3 for a T2 or T3 page (a T1 page carries 1.8x the bytes and
+// about the same compute), 0 for a dropped page, which is skipped.
 __device__ __forceinline__ uint32_t page_weight(int32_t e)
 {
     const int t = entry_tier(e);
@@ -808,8 +812,10 @@ constexpr int kGQ2 = 2 * kG;                          // heads per unit
 // products are page_logits'; the leaf terms go to 8 slots (slot i: head i ^ s).
 // T1: (w cos phi, w sin phi) times the 8 slots' query pairs, four 16-byte
 // rows in shared memory (the four token groups of the warp read the same
-// rows).  T2/T3: one 16-byte lookup in each of the two folded tables.  The 8-lane sum is a select-free reduce-scatter
-// (xor 4, 2, 1): after it lane s holds head s.
+// rows), summed slot pair by slot pair: slot i of lane s' goes straight to
+// lane s' ^ i.  T2/T3: one 16-byte lookup in each of the two folded tables,
+// then a select-free reduce-scatter (xor 4, 2, 1).  Either way lane s ends
+// with head s.
 template <int T>
 __device__ __forceinline__ void page_logits_pair(const uint8_t* pg, int lane, float (&lg)[4])
 {
