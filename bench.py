@@ -22,7 +22,13 @@ fits in L2, which its line states.
 
 value = token.heads/s = sum(seq_len) * H_q / time per step, aggregated over
 all ranks (weak scaling: every rank decodes its own batch, with no exchange
-between ranks; time is the max over ranks).
+between ranks; time is the max over ranks).  The line also gives the rate over
+kept tokens only (config.kept_token_heads_per_s).
+
+e2e = the same rate through host buffers: every step copies its inputs in from
+pinned host memory, makes the C-ABI call and copies out and lse back, then
+synchronises (one CUDA graph per step for the decode workloads; e2e_rdr also
+copies the step's new K/V rows in and appends them).
 
 --impl reference times the fp64 CPU oracle on the host cores, on a bounded
 sample of the same workload.
