@@ -323,13 +323,17 @@ __device__ inline int32_t cta_bound(int c, int32_t P, int n_cta)
     return (int32_t)(((int64_t)c * P) / n_cta);
 }
 
-// Work of a page by tier, for splitting a CTA's pages among its warps: 4 for
-// a T1 page, 3 for a T2 or T3 page (a T1 page carries 1.8x the bytes and
-// about the same compute), 0 for a dropped page, which is skipped.
+// Work of a page by tier, for splitting a CTA's pages among its warps, set
+// from measurements of each kernel: one query, T1 5 : T2/T3 6 (a T1 page
+// carries 1.8x the bytes but its leaves are cheaper than folded ones); a
+// pair, T1 5 : T2/T3 3 (its T1 leaves read query rows from shared memory).
+// A dropped page weighs 0 and is skipped.
+template <int NQ>
 __device__ __forceinline__ uint32_t page_weight(int32_t e)
 {
     const int t = entry_tier(e);
-    return t == 0 ? 0u : t == 1 ? 4u : 3u;
+    if (NQ == 1) return t == 0 ? 0u : t == 1 ? 5u : 6u;
+    return t == 0 ? 0u : t == 1 ? 5u : 3u;
 }
 
 // ------------------------------------------------------------- page work --
@@ -1090,7 +1094,7 @@ __global__ void __launch_bounds__(Layout<NQ>::kWarps * 32, 1) decode_kernel(Deco
         auto slice_start = [&](int k) -> int32_t { return pa + (int32_t)(((int64_t)n_seg * k) / kWarps); };
         {
             uint32_t sum = 0;
-            for (int32_t i = slice_start(w) + lane; i < slice_start(w + 1); i += 32) sum += page_weight(ptab[i]);
+            for (int32_t i = slice_start(w) + lane; i < slice_start(w + 1); i += 32) sum += page_weight<NQ>(ptab[i]);
             sum = __reduce_add_sync(full, sum);
             if (lane == 0) wsum[w] = sum;
         }
@@ -1183,7 +1187,7 @@ __global__ void __launch_bounds__(Layout<NQ>::kWarps * 32, 1) decode_kernel(Deco
                 const int32_t i1 = slice_start(j + 1);
                 for (int32_t base = slice_start(j); base < i1; base += 32) {
                     const int32_t i = base + lane;
-                    uint32_t c = i < i1 ? page_weight(ptab[i]) : 0u;
+                    uint32_t c = i < i1 ? page_weight<NQ>(ptab[i]) : 0u;
 #pragma unroll
                     for (int o = 1; o < 32; o <<= 1) {
                         const uint32_t y = __shfl_up_sync(full, c, o);
