@@ -89,3 +89,22 @@ def test_served_units_count_each_query_tokens_prefix():
     # n_q = 3: token 0 sees len - 2, token 1 len - 1, token 2 len
     per_seq = [max(5 - 2, 0) + 4 + 5, 0 + 0 + 1, 0, 38 + 39 + 40]
     assert bench.served_units(w, 3) == sum(per_seq) * 8
+
+
+def test_kept_units_counts_tokens_on_kept_pages():
+    """Kept-token rate: tokens on pages that are not dropped, times the query
+    heads per kv head, per query token (a later causal query sees one more
+    token).  Worked by hand on a two-sequence cache."""
+    w = W.make("ragged64", seq_lens=[40, 17], H_kv=2, H_q=8)
+    po = w.page_offsets               # sequence 0: pages 0..2, sequence 1: pages 3..4
+    w.tiers[:] = 1
+    w.tiers[0, po[0] + 1] = 0         # kv head 0, tokens 16..31 of sequence 0 dropped
+    w.tiers[1, po[1] + 1] = 0         # kv head 1, token 16 of sequence 1 dropped
+    # kv head 0: 40 - 16 + 17 = 41 tokens; kv head 1: 40 + 16 = 56; G = 4
+    assert bench.kept_units(w) == (41 + 56) * 4
+    # two causal queries: the first sees 39 and 16 tokens
+    first = ((39 - 16) + 16) + (39 + 16)
+    assert bench.kept_units(w, n_q=2) == (first + 41 + 56) * 4
+    # with nothing dropped it equals the served units
+    w.tiers[:] = 1
+    assert bench.kept_units(w) == bench.served_units(w)
