@@ -31,9 +31,10 @@ def test_library_exports_every_declared_symbol():
     # the binding covers the same names
     for n in names:
         assert n in _lib._EXPORTS or n in ("sphkv_last_error",), n
-    # the test-hook build (loaded only by tests) exports the same interface
-    T = ctypes.CDLL(build.TEST_LIB)
-    assert not [n for n in names if not hasattr(T, n)]
+    # the test-hook and checked builds (loaded only by tests) export the same interface
+    for path in (build.TEST_LIB, build.DEBUG_LIB):
+        T = ctypes.CDLL(path)
+        assert not [n for n in names if not hasattr(T, n)], path
 
 
 def test_host_helpers_agree_with_the_format():
